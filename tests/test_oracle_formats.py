@@ -1,0 +1,248 @@
+"""Pins of the CPU reference's number formats and quantizers (no GPU).
+
+Each test checks the reference against something other than itself: a
+library cast (ml_dtypes, torch), a worked example printed on the pages, a
+closed-form bound, or brute force over every code.
+"""
+import math
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+
+def _fp32_sweep(lo_exp, hi_exp, per_binade=4096, seed=0):
+    """Dense fp32 sample: every binade in [2**lo_exp, 2**hi_exp) at ``per_binade`` points
+    plus random bit patterns, both signs."""
+    rng = np.random.default_rng(seed)
+    vals = []
+    for e in range(lo_exp, hi_exp):
+        frac = np.arange(per_binade) / per_binade
+        vals.append((1.0 + frac) * 2.0 ** e)
+    v = np.concatenate(vals).astype(np.float32)
+    bits = rng.integers(0, 2 ** 32, size=200_000, dtype=np.uint64).astype(np.uint32)
+    r = bits.view(np.float32)
+    r = r[np.isfinite(r)]
+    r = r[(np.abs(r) >= 2.0 ** lo_exp) & (np.abs(r) < 2.0 ** hi_exp)]
+    v = np.concatenate([v, r, -v])
+    return v.astype(np.float32)
+
+
+# --------------------------------------------------------------------- bf16 / fp16
+
+def test_bf16_rn_matches_ml_dtypes_on_fp32():
+    x = _fp32_sweep(-40, 40)
+    # exact ties: bf16 value plus half an ulp, both parities of the kept bit
+    base = np.arange(0x0080, 0x7F00, 7, dtype=np.uint32) << 16   # normal exponents only
+    ties = (base | 0x8000).view(np.float32)
+    x = np.concatenate([x, ties, -ties, np.float32([0.0, -0.0, 1.0, -1.0])])
+    ours = O.bf16_rn(x)
+    lib = x.astype(ml_dtypes.bfloat16).astype(np.float32)
+    assert np.array_equal(ours.view(np.uint32), lib.view(np.uint32))
+
+
+def test_bf16_rn_fp64_is_nearest_even():
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal(50_000) * np.exp2(rng.integers(-20, 20, 50_000))
+    r = O.bf16_rn(x).astype(np.float64)
+    # neighbours on the bf16 grid: ulp = 2**(e-7) for |x| in [2**e, 2**(e+1))
+    e = np.floor(np.log2(np.abs(x)))
+    ulp = np.exp2(e - 7)
+    lo = np.floor(x / ulp) * ulp
+    hi = lo + ulp
+    d_lo, d_hi = x - lo, hi - x
+    m_lo = np.rint(lo / ulp).astype(np.int64)
+    want = np.where(d_lo < d_hi, lo, np.where(d_hi < d_lo, hi, np.where(m_lo % 2 == 0, lo, hi)))
+    assert np.array_equal(r, want)
+
+
+def test_fp16_rn_matches_torch():
+    x = _fp32_sweep(-24, 16)
+    ours = O.fp16_rn(x)
+    lib = torch.from_numpy(x).to(torch.float16).to(torch.float32).numpy()
+    assert np.array_equal(ours, lib)
+
+
+# --------------------------------------------------------------------- E4M3 / E2M1
+
+def test_e4m3_grid_is_the_format():
+    v = O.E4M3_VALUES
+    assert len(v) == 127 and v[0] == 0.0 and v[-1] == 448.0
+    assert v[1] == 2.0 ** -9 and v[8] == 2.0 ** -6           # min subnormal, min normal
+    lib = np.arange(127, dtype=np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float64)
+    assert np.array_equal(v, lib)
+
+
+def test_e4m3_rounding_matches_ml_dtypes():
+    x = _fp32_sweep(-12, 9)
+    x = x[np.abs(x) <= 448.0]
+    # every midpoint of the grid, and one fp32 ulp either side of it
+    mids = ((O.E4M3_VALUES[:-1] + O.E4M3_VALUES[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, np.nextafter(mids, 0), np.nextafter(mids, 1e9)]).astype(np.float32)
+    codes, vals = O.e4m3_rn_satfinite(x)
+    lib = x.astype(ml_dtypes.float8_e4m3fn)
+    assert np.array_equal(codes, lib.view(np.uint8))
+    assert np.array_equal(vals, lib.astype(np.float32))
+
+
+def test_e4m3_saturates():
+    codes, vals = O.e4m3_rn_satfinite(np.array([448.0, 460.0, 1e6, np.float32(3e38)]))
+    assert np.all(vals == 448.0) and np.all(codes == 0x7E)
+
+
+def test_e2m1_rounding_matches_ml_dtypes_and_ties():
+    x = _fp32_sweep(-6, 3)
+    x = x[np.abs(x) <= 6.0]
+    mids = ((O.E2M1_VALUES[:-1] + O.E2M1_VALUES[1:]) / 2).astype(np.float32)
+    x = np.concatenate([x, mids, -mids, np.nextafter(mids, 0), np.nextafter(mids, 9)])
+    codes, vals = O.e2m1_rn_satfinite(x)
+    lib = x.astype(ml_dtypes.float4_e2m1fn).astype(np.float32)
+    assert np.array_equal(vals, lib)
+    # ties go to the even code (reading 3)
+    t_in = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+    _, t_out = O.e2m1_rn_satfinite(t_in)
+    assert list(t_out) == [0.0, 1.0, 1.0, 2.0, 2.0, 4.0, 4.0]
+    # saturation at 6 and the kept sign of a small negative value
+    c, v = O.e2m1_rn_satfinite(np.array([7.0, -100.0, -0.1, 0.1, 0.0]))
+    assert list(v) == [6.0, -6.0, 0.0, 0.0, 0.0]
+    assert list(c) == [7, 15, 8, 0, 0]
+    assert np.signbit(v[2])
+
+
+# --------------------------------------------------------------------- INT4 g64
+
+def _int4_group(values):
+    g = np.zeros(64, np.float32)
+    g[: len(values)] = values
+    return g[None, :]
+
+
+def test_int4_worked_example(golden):
+    gd = golden("int4_rounding_example.txt")
+    grp = np.array(gd["group_with_outlier"], np.float32)
+    q = O.quantize_int4_g64(_int4_group(grp))
+    assert q["scale"][0, 0] == gd["step_with_outlier"]
+    assert list(q["q"][0, 1:len(grp)]) == gd["small_codes_with_outlier"]
+    # remove the large component: the remaining range is 1, the step is 1/7
+    small = grp.copy()
+    small[0] = np.float32(gd["remaining_range"])
+    q2 = O.quantize_int4_g64(_int4_group(small))
+    s = float(q2["scale"][0, 0])
+    assert abs(s - gd["step_without_outlier"]) <= 2.0 ** -14   # one fp16 half-ulp at 1/7
+    # with step 1/7 every one of the small elements gets a nonzero code
+    assert np.count_nonzero(q2["q"][0, 1:len(grp)]) == len(grp) - 1
+
+
+def test_int4_codes_are_argmin_over_all_codes():
+    rng = np.random.default_rng(3)
+    x = O.bf16_rn(rng.standard_normal((64, 256)) * np.exp2(rng.integers(-6, 6, (64, 1))))
+    q = O.quantize_int4_g64(x)
+    s = np.repeat(q["scale"], 64, axis=1).astype(np.float32)
+    t = (x / s).astype(np.float64)
+    cand = np.arange(-7, 8, dtype=np.float64)
+    d = np.abs(t[..., None] - cand)
+    best = d.min(axis=-1, keepdims=True)
+    ties = d == best
+    # among the nearest codes pick the even one (round half to even)
+    even = ties & (cand % 2 == 0)
+    pick = np.where(even.any(-1), cand[np.argmax(even, -1)], cand[np.argmax(ties, -1)])
+    assert np.array_equal(q["q"], pick)
+    assert q["q"].min() >= -7 and q["q"].max() <= 7
+    assert np.array_equal(O.int4_value(q["codes"]), q["q"])
+
+
+def test_int4_per_element_and_group_bound_eq9():
+    rng = np.random.default_rng(4)
+    x = O.bf16_rn(rng.standard_normal((32, 512)) * 0.02)
+    q = O.quantize_int4_g64(x)
+    s = np.repeat(q["scale"].astype(np.float64), 64, axis=1)
+    err = np.abs(x - s * q["q"])
+    unclamped = np.abs(x / s) <= 7.0
+    assert np.all(err[unclamped] <= s[unclamped] / 2 * (1 + 1e-7))
+    # eq.(9) per group with the group's own max: ||Z - Q(Z)||_F <= sqrt(N)/(2 qmax) max|Z|,
+    # loosened by the fp16 rounding of the scale (relative 2**-11).
+    e = (x - s * q["q"]).reshape(32, 8, 64)
+    lhs = np.sqrt((e ** 2).sum(-1))
+    rhs = math.sqrt(64) / (2 * 7) * np.abs(x.reshape(32, 8, 64)).max(-1) * (1 + 2.0 ** -10)
+    assert np.all(lhs <= rhs)
+
+
+def test_int4_zero_group_and_scale_precision():
+    x = np.zeros((2, 128), np.float32)
+    x[1, 64:] = 3.0
+    q = O.quantize_int4_g64(x)
+    assert np.all(q["q"][0] == 0) and q["scale"][0, 0] == 0
+    assert q["scale"][1, 1] == O.fp16_rn(np.float32(3.0) / np.float32(7.0))
+    assert np.all(q["q"][1, 64:] == 7)
+
+
+# --------------------------------------------------------------------- NVFP4 g16
+
+def test_nvfp4_scales_and_codes_are_nearest():
+    rng = np.random.default_rng(5)
+    x = O.bf16_rn(rng.standard_normal((48, 256)) * np.exp2(rng.integers(-8, 4, (48, 1))))
+    g = O.pow2_global_scale(np.abs(x).max())
+    q = O.quantize_nvfp4_g16(x, g)
+    a = np.abs(x.reshape(48, 16, 16)).max(-1)
+    t = ((a / np.float32(6.0)).astype(np.float32) / np.float32(g)).astype(np.float32)
+    # scale = nearest E4M3 to t (brute force over the whole grid, ties to even code)
+    d = np.abs(t[..., None].astype(np.float64) - O.E4M3_VALUES)
+    best = d.min(-1, keepdims=True)
+    ties = d == best
+    even = ties & (np.arange(127) % 2 == 0)
+    want = np.where(even.any(-1), np.argmax(even, -1), np.argmax(ties, -1))
+    assert np.array_equal(q["scale_bits"].astype(np.int64), want)
+    # codes = nearest E2M1 value of x / (s g), ties to even
+    den = np.repeat((q["scale"] * np.float32(g)).astype(np.float32), 16, axis=1)
+    v = (x / den).astype(np.float64)
+    grid = np.concatenate([-O.E2M1_VALUES[::-1], O.E2M1_VALUES])
+    dv = np.abs(np.minimum(np.abs(v), 6.0)[..., None] - O.E2M1_VALUES)
+    assert np.all(np.abs(np.abs(q["q"]) - np.minimum(np.abs(v), 6.0)) <= dv.min(-1) + 1e-12)
+    assert set(np.unique(q["q"])).issubset(set(grid))
+    assert np.array_equal(np.sign(q["q"][q["q"] != 0]), np.sign(v[q["q"] != 0]))
+
+
+def test_nvfp4_dequant_error_bound():
+    rng = np.random.default_rng(6)
+    x = O.bf16_rn(rng.standard_normal((16, 1024)) * 0.05)
+    g = O.pow2_global_scale(np.abs(x).max())
+    q = O.quantize_nvfp4_g16(x, g)
+    deq = O.dequantize("nvfp4", q)
+    s = np.repeat(q["scale"].astype(np.float64) * g, 16, axis=1)
+    # the E2M1 grid gap is at most 2 (between 4 and 6), so half a gap times s,
+    # plus the clamp when the rounded scale is below a/6
+    a = np.repeat(np.abs(x.reshape(16, 64, 16)).max(-1), 16, axis=1)
+    err = np.abs(x - deq)
+    assert np.all(err <= s * 1.0 + np.maximum(a - 6 * s, 0) + 1e-12)
+
+
+def test_pow2_global_scale():
+    for amax in (1e-3, 0.02, 0.5, 3.0, 37.0, 1000.0):
+        g = O.pow2_global_scale(amax)
+        assert math.log2(g) == int(math.log2(g))
+        assert 0.5 < amax / (6 * 448 * g) <= 1.0
+    assert O.pow2_global_scale(0.0) == 1.0
+
+
+# --------------------------------------------------------------------- planted mistakes
+
+def test_planted_sign_drop_in_e2m1_is_caught(monkeypatch):
+    """A quantizer that loses the sign must fail the library cross-check."""
+    good = O.e2m1_rn_satfinite
+
+    def bad(x):
+        c, v = good(np.abs(x))
+        return c, v
+    monkeypatch.setattr(O, "e2m1_rn_satfinite", bad)
+    x = np.array([-1.0, -3.0, 2.0], np.float32)
+    _, v = O.e2m1_rn_satfinite(x)
+    assert not np.array_equal(v, x.astype(ml_dtypes.float4_e2m1fn).astype(np.float32))
+
+
+def test_planted_round_half_up_is_caught():
+    """Rounding half away from zero (instead of to even) breaks the argmin pin on ties."""
+    t = np.array([0.5, 1.5, 2.5, -2.5], np.float64)
+    assert not np.array_equal(np.floor(t + 0.5), np.rint(t))
