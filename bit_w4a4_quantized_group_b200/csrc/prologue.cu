@@ -1,0 +1,350 @@
+// Prologue kernel: smoothing divide, group quantization and low-rank down
+// projection in one read of X.
+//
+// "SVDQuant 阅读笔记：用少量高精度计算保护 4-bit 扩散模型", §6.1 "算法 2"
+// steps 1-3: read a tile of the high-precision activations once, reuse it for
+// Z = X_hat L1 and for the 4-bit quantization (codes + scales).  The smoothing
+// divide is X D^-1 of §3.1 eq.(3); the quantizers are eq.(1) (INT4 g64,
+// 16-bit scale) and NVFP4 g16 with E4M3 scales (§2.2, §8).
+//
+// Design (B200): HBM-bound.  A dedicated producer warp streams 32-row x
+// 256-column tiles of X (and the matching 256 columns of L1 and lambda) into
+// a shared-memory ring with TMA; eight compute warps each own a 16-row x
+// 64-column box of every tile.  X_hat is formed in registers in the
+// m16n8k16 fragment layout so that the same registers feed the bf16 tensor-
+// core MMA for Z and the quantizer; codes are staged per warp in shared
+// memory and written back as 16-byte row segments.  Z partials of the four
+// warps that share a row strip are summed in a fixed order (deterministic).
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+#include "svdq_device.cuh"
+
+namespace svdq {
+
+namespace {
+
+constexpr int kProThreads = 288;      // 8 compute warps + 1 producer warp
+constexpr int kProRows = 32;          // rows per CTA
+constexpr int kProCols = 256;         // columns per pipeline stage (4 boxes of 64)
+constexpr uint32_t kXBoxBytes = kProRows * 128;   // 32 rows x 64 bf16
+
+struct ProSmemLayout {
+  uint32_t x_off, l1_off, lam_off, stage_bytes;
+};
+
+__host__ __device__ inline ProSmemLayout pro_layout(int rank) {
+  ProSmemLayout L;
+  L.x_off = 0;
+  L.l1_off = 4 * kXBoxBytes;                       // 16 KB
+  L.lam_off = L.l1_off + 4u * 128u * rank;         // 4 boxes of r rows x 128 B
+  uint32_t sz = L.lam_off + kProCols * 4;          // 1 KB of lambda
+  L.stage_bytes = (sz + 1023u) & ~1023u;
+  return L;
+}
+
+__device__ __forceinline__ float bf16lo(uint32_t v) { return __uint_as_float(v << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<uint32_t*>(&h);
+}
+
+template <int FMT, int RANK>
+__global__ void __launch_bounds__(kProThreads, 1)
+    prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_l1,
+                    ProParams p) {
+  constexpr int NT = RANK / 8;                  // n8 tiles of Z
+  const ProSmemLayout L = pro_layout(RANK);
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int S = p.stages;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * L.stage_bytes);
+  uint64_t* empty = full + S;
+  uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // 8 warps x 512 B code staging
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(cstage + 8 * 512);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int m0 = blockIdx.x * kProRows;
+  const int nkt = (p.K + kProCols - 1) / kProCols;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 8);
+    }
+    *abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncthreads();
+
+  if (warp == 8) {
+    // ---------------------------------------------------------------- producer
+    if (ptx::elect_one()) {
+      ptx::prefetch_tmap(&tmap_x);
+      if (RANK > 0) ptx::prefetch_tmap(&tmap_l1);
+      for (int kt = 0; kt < nkt; ++kt) {
+        const int s = kt % S;
+        const uint32_t ph = (kt / S) & 1;
+        if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
+        const int col0 = kt * kProCols;
+        const int cols = min(kProCols, p.K - col0);
+        const int nbox = cols / 64;
+        uint32_t bytes = nbox * (kXBoxBytes + 128u * RANK) + (p.lam ? cols * 4u : 0u);
+        ptx::mbar_arrive_expect_tx(&full[s], bytes);
+        uint8_t* st = smem + s * L.stage_bytes;
+        for (int b = 0; b < nbox; ++b) {
+          ptx::tma_load_2d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], col0 + b * 64, m0);
+          if (RANK > 0) ptx::tma_load_2d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], col0 + b * 64, 0);
+        }
+        if (p.lam) ptx::bulk_load(st + L.lam_off, p.lam + col0, cols * 4u, &full[s]);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ---------------------------------------------------------------- compute warps
+    const int strip = warp & 1;         // rows 16*strip .. 16*strip+15 of the CTA tile
+    const int phase = warp >> 1;        // 64-column box of every stage
+    const int g = lane >> 2, tig = lane & 3;
+    const int row_a = m0 + strip * 16 + g;   // rows of this thread's fragments
+    const int row_b = row_a + 8;
+    float acc[NT > 0 ? NT : 1][4];
+#pragma unroll
+    for (int i = 0; i < (NT > 0 ? NT : 1); ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
+    uint8_t* cst = cstage + warp * 512;
+    const int K2 = p.K / 2;
+    const float gs = p.gscale;
+    bool ok = true;
+
+    for (int kt = 0; kt < nkt && ok; ++kt) {
+      const int s = kt % S;
+      const uint32_t ph = (kt / S) & 1;
+      if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
+      const int col0 = kt * kProCols + phase * 64;
+      if (col0 < p.K) {
+        const uint8_t* st = smem + s * L.stage_bytes;
+        const uint32_t xbox = ptx::smem_u32(st + L.x_off + phase * kXBoxBytes);
+        const uint32_t l1box = ptx::smem_u32(st + L.l1_off + phase * 128 * RANK);
+        const float* lam_s = reinterpret_cast<const float*>(st + L.lam_off) + phase * 64;
+        float xv[4][8];                 // X_hat values: [k16 tile][row g: 0..3, row g+8: 4..7]
+        uint32_t sc_pack_a = 0, sc_pack_b = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          uint32_t a[4];
+          {
+            const int r = strip * 16 + (lane & 7) + ((lane >> 3) & 1) * 8;
+            const int ch = 2 * j + (lane >> 4);
+            ptx::ldmatrix_x4(xbox + r * 128 + ((ch ^ (r & 7)) << 4), a[0], a[1], a[2], a[3]);
+          }
+          const int c0 = j * 16 + tig * 2;
+          // smoothing divide X / lambda (IEEE fp32), one rounding to bf16
+          float l0 = 1.f, l1 = 1.f, l8 = 1.f, l9 = 1.f;
+          if (p.lam) { l0 = lam_s[c0]; l1 = lam_s[c0 + 1]; l8 = lam_s[c0 + 8]; l9 = lam_s[c0 + 9]; }
+          uint32_t ah[4];
+          {
+            float x0 = bf16lo(a[0]) / l0, x1 = bf16hi(a[0]) / l1;   // row g,   cols c0, c0+1
+            float x2 = bf16lo(a[1]) / l0, x3 = bf16hi(a[1]) / l1;   // row g+8, cols c0, c0+1
+            float x4 = bf16lo(a[2]) / l8, x5 = bf16hi(a[2]) / l9;   // row g,   cols c0+8, c0+9
+            float x6 = bf16lo(a[3]) / l8, x7 = bf16hi(a[3]) / l9;   // row g+8, cols c0+8, c0+9
+            ah[0] = pack_bf16x2(x0, x1);
+            ah[1] = pack_bf16x2(x2, x3);
+            ah[2] = pack_bf16x2(x4, x5);
+            ah[3] = pack_bf16x2(x6, x7);
+          }
+          xv[j][0] = bf16lo(ah[0]); xv[j][1] = bf16hi(ah[0]);
+          xv[j][2] = bf16lo(ah[2]); xv[j][3] = bf16hi(ah[2]);
+          xv[j][4] = bf16lo(ah[1]); xv[j][5] = bf16hi(ah[1]);
+          xv[j][6] = bf16lo(ah[3]); xv[j][7] = bf16hi(ah[3]);
+          // low-rank down projection on the tensor cores
+#pragma unroll
+          for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
+            uint32_t b[4];
+            const int n = nt2 * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
+            const int ch = 2 * j + ((lane >> 3) & 1);
+            ptx::ldmatrix_x4(l1box + n * 128 + ((ch ^ (n & 7)) << 4), b[0], b[1], b[2], b[3]);
+            ptx::mma_bf16_16816(acc[2 * nt2], ah, b[0], b[1]);
+            ptx::mma_bf16_16816(acc[2 * nt2 + 1], ah, b[2], b[3]);
+          }
+          if (FMT == kFmtNvfp4) {
+            // one 16-element group per row per k16 tile
+            float ma = fmaxf(fmaxf(fabsf(xv[j][0]), fabsf(xv[j][1])), fmaxf(fabsf(xv[j][2]), fabsf(xv[j][3])));
+            float mb = fmaxf(fmaxf(fabsf(xv[j][4]), fabsf(xv[j][5])), fmaxf(fabsf(xv[j][6]), fabsf(xv[j][7])));
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+            const uint32_t sa = ptx::cvt_e4m3((ma / 6.0f) / gs);
+            const uint32_t sb = ptx::cvt_e4m3((mb / 6.0f) / gs);
+            const float da = ptx::e4m3_to_f32(sa) * gs;
+            const float db = ptx::e4m3_to_f32(sb) * gs;
+            uint32_t qa0 = 0, qa1 = 0, qb0 = 0, qb1 = 0;
+            if (da > 0.f) {
+              qa0 = ptx::cvt_e2m1x2(xv[j][0] / da, xv[j][1] / da);
+              qa1 = ptx::cvt_e2m1x2(xv[j][2] / da, xv[j][3] / da);
+            }
+            if (db > 0.f) {
+              qb0 = ptx::cvt_e2m1x2(xv[j][4] / db, xv[j][5] / db);
+              qb1 = ptx::cvt_e2m1x2(xv[j][6] / db, xv[j][7] / db);
+            }
+            cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(qa0);
+            cst[g * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(qa1);
+            cst[(g + 8) * 32 + j * 8 + tig] = static_cast<uint8_t>(qb0);
+            cst[(g + 8) * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(qb1);
+            sc_pack_a |= sa << (8 * j);
+            sc_pack_b |= sb << (8 * j);
+          }
+        }
+        if (FMT == kFmtInt4) {
+          // one 64-element group per row per box
+          float ma = 0.f, mb = 0.f;
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              ma = fmaxf(ma, fabsf(xv[j][e]));
+              mb = fmaxf(mb, fabsf(xv[j][4 + e]));
+            }
+          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+          mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+          mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+          const __half ha = __float2half_rn(fminf(ma / 7.0f, 65504.0f));
+          const __half hb = __float2half_rn(fminf(mb / 7.0f, 65504.0f));
+          const float fa = __half2float(ha), fb = __half2float(hb);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t q[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float den = (e < 4) ? fa : fb;
+              int v = 0;
+              if (den > 0.f) v = max(-7, min(7, __float2int_rn(xv[j][e] / den)));
+              q[e] = static_cast<uint32_t>(v) & 0xFu;
+            }
+            cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(q[0] | (q[1] << 4));
+            cst[g * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(q[2] | (q[3] << 4));
+            cst[(g + 8) * 32 + j * 8 + tig] = static_cast<uint8_t>(q[4] | (q[5] << 4));
+            cst[(g + 8) * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(q[6] | (q[7] << 4));
+          }
+          if (tig == 0) {
+            const int grp = col0 / 64;
+            __half* sc = reinterpret_cast<__half*>(p.scales);
+            sc[static_cast<size_t>(grp) * p.Mpad + row_a] = ha;
+            sc[static_cast<size_t>(grp) * p.Mpad + row_b] = hb;
+          }
+        } else {
+          if (tig == 0) {
+            // 4 consecutive E4M3 bytes of the 128x4 blocked layout per row
+            const int grp4 = col0 / 64;              // index of the 4-group block along K
+            uint8_t* sc = reinterpret_cast<uint8_t*>(p.scales);
+            const size_t ba = (static_cast<size_t>(row_a / 128) * (p.K / 64) + grp4) * 512 +
+                              (row_a % 32) * 16 + ((row_a % 128) / 32) * 4;
+            const size_t bb = (static_cast<size_t>(row_b / 128) * (p.K / 64) + grp4) * 512 +
+                              (row_b % 32) * 16 + ((row_b % 128) / 32) * 4;
+            *reinterpret_cast<uint32_t*>(sc + ba) = sc_pack_a;
+            *reinterpret_cast<uint32_t*>(sc + bb) = sc_pack_b;
+          }
+        }
+        __syncwarp();
+        // 16 rows x 32 bytes of codes -> global, one 16-byte segment per lane
+        {
+          const int r = lane >> 1, h = lane & 1;
+          const int row = m0 + strip * 16 + r;
+          const uint4 v = *reinterpret_cast<const uint4*>(cst + r * 32 + h * 16);
+          if (row < p.M) *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * K2 + col0 / 2 + h * 16) = v;
+        }
+        __syncwarp();
+      }
+      if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    }
+
+    // ---------------------------------------------------------------- Z = X_hat L1^T
+    if (NT > 0) {
+      __syncthreads_compute(ok);
+      float* zbuf = reinterpret_cast<float*>(smem);       // [phase][strip][16][RANK]
+      float* zb = zbuf + ((phase * 2 + strip) * 16) * RANK;
+#pragma unroll
+      for (int nt = 0; nt < NT; ++nt) {
+        const int c = nt * 8 + tig * 2;
+        zb[g * RANK + c] = acc[nt][0];
+        zb[g * RANK + c + 1] = acc[nt][1];
+        zb[(g + 8) * RANK + c] = acc[nt][2];
+        zb[(g + 8) * RANK + c + 1] = acc[nt][3];
+      }
+      __syncthreads_compute(ok);
+      // warps of phase 0 sum the four partials in phase order and store bf16
+      if (phase == 0) {
+        for (int idx = lane; idx < 16 * RANK / 2; idx += 32) {
+          const int r = (idx * 2) / (RANK > 0 ? RANK : 1), c = (idx * 2) % (RANK > 0 ? RANK : 1);
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int ph = 0; ph < 4; ++ph) {
+            const float* src = zbuf + ((ph * 2 + strip) * 16 + r) * RANK + c;
+            s0 += src[0];
+            s1 += src[1];
+          }
+          const int row = m0 + strip * 16 + r;
+          if (row < p.M) {
+            __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
+            *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * RANK + c) = v;
+          }
+        }
+      }
+    }
+  }
+}
+
+}  // namespace
+
+size_t prologue_smem_bytes(int rank, int stages) {
+  const ProSmemLayout L = pro_layout(rank);
+  return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + 8 * 512 + 16;
+}
+
+int prologue_stages(int rank) {
+  const ProSmemLayout L = pro_layout(rank);
+  int s = static_cast<int>((200u * 1024u) / L.stage_bytes);
+  if (s > 4) s = 4;
+  if (s < 2) s = 2;
+  return s;
+}
+
+template <int FMT, int RANK>
+static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
+                              cudaStream_t stream) {
+  const size_t smem = prologue_smem_bytes(RANK, p.stages);
+  auto kern = prologue_kernel<FMT, RANK>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  const int grid = p.Mpad / kProRows;
+  kern<<<grid, kProThreads, smem, stream>>>(tx, tl1, p);
+  return cudaGetLastError();
+}
+
+template <int FMT>
+static cudaError_t launch_pro_rank(const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
+                                   cudaStream_t s) {
+  switch (p.rank) {
+    case 0: return launch_pro<FMT, 0>(tx, tl1, p, s);
+    case 16: return launch_pro<FMT, 16>(tx, tl1, p, s);
+    case 32: return launch_pro<FMT, 32>(tx, tl1, p, s);
+    case 48: return launch_pro<FMT, 48>(tx, tl1, p, s);
+    case 64: return launch_pro<FMT, 64>(tx, tl1, p, s);
+    case 80: return launch_pro<FMT, 80>(tx, tl1, p, s);
+    case 96: return launch_pro<FMT, 96>(tx, tl1, p, s);
+    case 112: return launch_pro<FMT, 112>(tx, tl1, p, s);
+    case 128: return launch_pro<FMT, 128>(tx, tl1, p, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
+                            cudaStream_t s) {
+  return fmt == kFmtNvfp4 ? launch_pro_rank<kFmtNvfp4>(tx, tl1, p, s) : launch_pro_rank<kFmtInt4>(tx, tl1, p, s);
+}
+
+}  // namespace svdq

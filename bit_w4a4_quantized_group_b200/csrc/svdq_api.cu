@@ -1,0 +1,228 @@
+// C ABI of libsvdq: argument checks, TMA descriptor set-up and launches.
+// The operations are specified in include/svdq.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <cudaTypedefs.h>
+
+#include <cstdint>
+#include <cstring>
+#include <mutex>
+
+#include "svdq.h"
+#include "svdq_device.cuh"
+#include "svdq_internal.h"
+
+namespace svdq {
+
+__device__ int g_device_error = 0;   // the library's one piece of device state (per device)
+
+namespace {
+
+thread_local int t_last_launch_count = 0;
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 2-D row-major tensor [outer][inner] of `elem` bytes per element, tiled with a
+// box of box_inner x box_outer elements and 128-byte swizzle.
+bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t inner,
+               uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {inner, outer};
+  cuuint64_t strides[1] = {inner * static_cast<uint64_t>(elem)};
+  cuuint32_t box[2] = {box_inner, box_outer};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int device_sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cache[64] = {0};
+  if (dev < 0 || dev >= 64) return 0;
+  if (cache[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+    cache[dev] = n;
+  }
+  return cache[dev];
+}
+
+int* device_error_word() {
+  void* p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_device_error) != cudaSuccess) return nullptr;
+  return static_cast<int*>(p);
+}
+
+size_t scale_bytes(svdq_format fmt, int64_t rows, int64_t K) {
+  const int64_t rp = (rows + 127) / 128 * 128;
+  return fmt == SVDQ_FMT_NVFP4_G16 ? static_cast<size_t>(rp * (K / 16)) : static_cast<size_t>(rp * (K / 64) * 2);
+}
+
+}  // namespace
+}  // namespace svdq
+
+using namespace svdq;
+
+extern "C" const char* svdq_status_string(svdq_status s) {
+  switch (s) {
+    case SVDQ_OK: return "ok";
+    case SVDQ_ERR_INVALID_ARG: return "invalid argument";
+    case SVDQ_ERR_UNSUPPORTED: return "unsupported";
+    case SVDQ_ERR_CUDA: return "CUDA error";
+    case SVDQ_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+extern "C" svdq_status svdq_buffer_sizes(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank,
+                                         svdq_sizes* out) {
+  svdq_status st = check_dims(fmt, M, N, K, rank);
+  if (st != SVDQ_OK) return st;
+  if (!out) return SVDQ_ERR_INVALID_ARG;
+  out->x = static_cast<size_t>(M * K * 2);
+  out->a_codes = static_cast<size_t>(M * K / 2);
+  out->a_scales = scale_bytes(fmt, M, K);
+  out->z = static_cast<size_t>(M * rank * 2);
+  out->w_codes = static_cast<size_t>(N * K / 2);
+  out->w_scales = scale_bytes(fmt, N, K);
+  out->l1 = static_cast<size_t>(int64_t(rank) * K * 2);
+  out->l2 = static_cast<size_t>(N * rank * 2);
+  out->bias = static_cast<size_t>(N * 2);
+  out->y = static_cast<size_t>(M * N * 2);
+  return SVDQ_OK;
+}
+
+extern "C" int svdq_last_launch_count(void) { return t_last_launch_count; }
+
+extern "C" svdq_status svdq_get_last_device_error(void* cuda_stream, int* site) {
+  if (site) *site = 0;
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return SVDQ_ERR_CUDA;
+  int* w = device_error_word();
+  if (!w) return SVDQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpy(&v, w, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (v != 0) {
+    const int zero = 0;
+    if (cudaMemcpy(w, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess) return SVDQ_ERR_CUDA;
+    if (site) *site = v;
+    return SVDQ_ERR_TIMEOUT;
+  }
+  return SVDQ_OK;
+}
+
+extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M, int64_t K, int rank,
+                                                      const void* X_bf16, const float* lambda, float act_gscale,
+                                                      const void* L1_bf16, void* a_codes, void* a_scales,
+                                                      void* Z_bf16, void* cuda_stream) {
+  t_last_launch_count = 0;
+  svdq_status st = check_dims(fmt, M, 128, K, rank);
+  if (st != SVDQ_OK) return st;
+  if (!X_bf16 || !a_codes || !a_scales) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(X_bf16) || !aligned16(a_codes) || !aligned16(a_scales)) return SVDQ_ERR_INVALID_ARG;
+  if (lambda && !aligned16(lambda)) return SVDQ_ERR_INVALID_ARG;
+  if (rank > 0 && (!L1_bf16 || !Z_bf16 || !aligned16(L1_bf16) || !aligned16(Z_bf16))) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_positive(act_gscale)) return SVDQ_ERR_INVALID_ARG;
+  if (fmt == SVDQ_FMT_INT4_G64 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
+
+  CUtensorMap tx, tl1;
+  if (!make_tmap(&tx, X_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64, 32)) return SVDQ_ERR_CUDA;
+  if (rank > 0) {
+    if (!make_tmap(&tl1, L1_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rank, 64, rank)) return SVDQ_ERR_CUDA;
+  } else {
+    tl1 = tx;
+  }
+  ProParams p{};
+  p.M = static_cast<int>(M);
+  p.K = static_cast<int>(K);
+  p.rank = rank;
+  p.Mpad = static_cast<int>((M + 127) / 128 * 128);
+  p.stages = prologue_stages(rank);
+  p.lam = lambda;
+  p.gscale = act_gscale;
+  p.codes = static_cast<uint8_t*>(a_codes);
+  p.scales = a_scales;
+  p.Z = static_cast<__nv_bfloat16*>(Z_bf16);
+  p.err = device_error_word();
+  if (!p.err) return SVDQ_ERR_CUDA;
+  cudaError_t e = launch_prologue(fmt == SVDQ_FMT_NVFP4_G16 ? kFmtNvfp4 : kFmtInt4, tx, tl1, p,
+                                  static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  t_last_launch_count = 1;
+  return SVDQ_OK;
+}
+
+extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank,
+                                                 const void* a_codes, const void* a_scales, float act_gscale,
+                                                 const void* w_codes, const void* w_scales, float w_gscale,
+                                                 const void* Z_bf16, const void* L2_bf16, const void* bias_bf16,
+                                                 void* Y_bf16, void* cuda_stream) {
+  t_last_launch_count = 0;
+  svdq_status st = check_dims(fmt, M, N, K, rank);
+  if (st != SVDQ_OK) return st;
+  if (!a_codes || !a_scales || !w_codes || !w_scales || !Y_bf16) return SVDQ_ERR_INVALID_ARG;
+  if (!aligned16(a_codes) || !aligned16(a_scales) || !aligned16(w_codes) || !aligned16(w_scales) ||
+      !aligned16(Y_bf16))
+    return SVDQ_ERR_INVALID_ARG;
+  if (bias_bf16 && !aligned16(bias_bf16)) return SVDQ_ERR_INVALID_ARG;
+  if (rank > 0 && (!Z_bf16 || !L2_bf16 || !aligned16(Z_bf16) || !aligned16(L2_bf16))) return SVDQ_ERR_INVALID_ARG;
+  if (!is_pow2_positive(act_gscale) || !is_pow2_positive(w_gscale)) return SVDQ_ERR_INVALID_ARG;
+  if (fmt == SVDQ_FMT_INT4_G64 && (act_gscale != 1.0f || w_gscale != 1.0f)) return SVDQ_ERR_INVALID_ARG;
+
+  const int sms = device_sm_count();
+  if (sms <= 0) return SVDQ_ERR_CUDA;
+  GemmParams p{};
+  p.M = static_cast<int>(M);
+  p.N = static_cast<int>(N);
+  p.K = static_cast<int>(K);
+  p.rank = rank;
+  p.Mpad = static_cast<int>((M + 127) / 128 * 128);
+  p.Npad = static_cast<int>((N + 127) / 128 * 128);
+  p.out_scale = act_gscale * w_gscale;
+  p.a_codes = static_cast<const uint8_t*>(a_codes);
+  p.w_codes = static_cast<const uint8_t*>(w_codes);
+  p.a_scales = static_cast<const uint8_t*>(a_scales);
+  p.w_scales = static_cast<const uint8_t*>(w_scales);
+  p.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
+  p.Y = static_cast<__nv_bfloat16*>(Y_bf16);
+  p.err = device_error_word();
+  if (!p.err) return SVDQ_ERR_CUDA;
+
+  CUtensorMap tz, tl2;
+  cudaError_t e;
+  if (fmt == SVDQ_FMT_NVFP4_G16) {
+    p.tiles_m = static_cast<int>((M + 127) / 128);
+    p.tiles_n = static_cast<int>((N + 255) / 256);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    CUtensorMap ta, tb;
+    if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) return SVDQ_ERR_CUDA;
+    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 256)) return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+      if (!make_tmap(&tz, Z_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, M, 64, 128)) return SVDQ_ERR_CUDA;
+      if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 256)) return SVDQ_ERR_CUDA;
+    } else {
+      tz = ta;
+      tl2 = tb;
+    }
+    e = launch_gemm_nvfp4(ta, tb, tz, tl2, p, sms, static_cast<cudaStream_t>(cuda_stream));
+  } else {
+    return SVDQ_ERR_UNSUPPORTED;
+  }
+  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  t_last_launch_count = 1;
+  return SVDQ_OK;
+}

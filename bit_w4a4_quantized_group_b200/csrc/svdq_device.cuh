@@ -1,0 +1,90 @@
+// Device-side declarations shared by the kernels of libsvdq.
+#pragma once
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <cstdint>
+
+#include "ptx.cuh"
+
+namespace svdq {
+
+constexpr int kFmtNvfp4 = 1;
+constexpr int kFmtInt4 = 2;
+
+// Codes recorded in the device error word when a bounded wait runs out.
+enum : int {
+  kErrSiteProEmpty = 1,
+  kErrSiteProFull = 2,
+  kErrSiteGemmEmpty = 11,
+  kErrSiteGemmFull = 12,
+  kErrSiteGemmAccEmpty = 13,
+  kErrSiteGemmAccFull = 14,
+  kErrSiteGemmConvEmpty = 15,
+  kErrSiteGemmConvFull = 16,
+};
+
+// A wait gives up after this many nanoseconds (~1 s); legitimate waits here
+// last microseconds.
+constexpr uint64_t kWaitLimitNs = 1000000000ull;
+
+// Parity wait on an mbarrier with a time limit.  On time-out the first waiter
+// records its site in the device error word, raises the CTA's abort flag and
+// returns false; waiters that see the abort flag return false as well.
+__device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                             int* err, int site) {
+  const uint32_t a = ptx::smem_u32(bar);
+  if (ptx::mbar_try_wait(a, parity)) return true;
+  const uint64_t t0 = ptx::globaltimer();
+  uint32_t spins = 0;
+  while (true) {
+    if (ptx::mbar_try_wait(a, parity)) return true;
+    if ((++spins & 63u) == 0) {
+      if (*abort_flag) return false;
+      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+        atomicCAS(err, 0, site);
+        *abort_flag = 1;
+        return false;
+      }
+    }
+  }
+}
+
+// Barrier over the 256 compute threads of the prologue (named barrier 1).
+__device__ __forceinline__ void __syncthreads_compute(bool) { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+
+struct ProParams {
+  int M, K, rank, Mpad, stages;
+  const float* lam;          // nullable
+  float gscale;              // activation tensor scale (NVFP4), 1 for INT4
+  uint8_t* codes;            // [M][K/2]
+  void* scales;              // format-specific layout
+  __nv_bfloat16* Z;          // [M][rank]
+  int* err;                  // device error word
+};
+
+struct GemmParams {
+  int M, N, K, rank;
+  int Mpad, Npad;
+  float out_scale;           // act_gscale * w_gscale
+  const uint8_t* a_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Mpad]
+  const uint8_t* w_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Npad]
+  const uint8_t* a_codes;    // [M][K/2]
+  const uint8_t* w_codes;    // [N][K/2]
+  const __nv_bfloat16* bias; // nullable
+  __nv_bfloat16* Y;          // [M][N]
+  int* err;
+  int num_tiles, tiles_m, tiles_n;
+};
+
+size_t prologue_smem_bytes(int rank, int stages);
+int prologue_stages(int rank);
+cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
+                            cudaStream_t s);
+
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
+                              const CUtensorMap& tl2, const GemmParams& p, int num_sms, cudaStream_t s);
+cudaError_t launch_gemm_int4(const CUtensorMap& tz, const CUtensorMap& tl2, const GemmParams& p, int num_sms,
+                             cudaStream_t s);
+
+}  // namespace svdq

@@ -251,7 +251,14 @@ def pow2_global_scale(amax: float) -> float:
     amax = float(amax)
     if not amax > 0.0:
         return 1.0
-    return float(2.0 ** math.ceil(math.log2(amax / (NVFP4_QMAX * E4M3_MAX))))
+    lim = NVFP4_QMAX * E4M3_MAX
+    e = math.frexp(amax / lim)[1]
+    # exact comparisons decide the boundary cases (amax / lim a power of two)
+    while lim * 2.0 ** (e - 1) >= amax:
+        e -= 1
+    while lim * 2.0 ** e < amax:
+        e += 1
+    return float(2.0 ** e)
 
 
 def quantize_int4_g64(x: np.ndarray):

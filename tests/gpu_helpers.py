@@ -1,0 +1,88 @@
+"""Helpers of the GPU parity tests: run the library through the C ABI on
+seeded inputs and bring results back in canonical form."""
+import numpy as np
+import torch
+
+from bit_w4a4_quantized_group_b200 import binding as B
+
+from layouts import (bf16_bits_to_f32, f32_to_bf16_bits_exact, nvfp4_scale_offsets, scales_canonical,
+                     scales_padding, unpack_codes)
+
+
+def dev_bf16(x: np.ndarray) -> torch.Tensor:
+    """float32 array of exact bf16 values -> device bf16 tensor (bit exact)."""
+    bits = f32_to_bf16_bits_exact(np.ascontiguousarray(x, np.float32))
+    return torch.from_numpy(bits.view(np.int16)).cuda().view(torch.bfloat16)
+
+
+def host_bf16(t: torch.Tensor) -> np.ndarray:
+    return bf16_bits_to_f32(t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16))
+
+
+def check_device_error():
+    torch.cuda.synchronize()
+    st, site = B.svdq_get_last_device_error(None)
+    assert st == B.SVDQ_OK, f"device error status {st} at wait site {site}"
+
+
+def run_prologue(fmt, X, lam, gx, L1_rk, fill=0x5A):
+    M, K = X.shape
+    r = 0 if L1_rk is None else L1_rk.shape[0]
+    sz = B.svdq_buffer_sizes(fmt, M, 128, K, r)
+    Xd = dev_bf16(X)
+    lam_d = None if lam is None else torch.from_numpy(np.ascontiguousarray(lam, np.float32)).cuda()
+    L1d = dev_bf16(L1_rk) if r > 0 else None
+    codes = torch.full((sz.a_codes,), fill, dtype=torch.uint8, device="cuda")
+    scales = torch.full((sz.a_scales,), fill, dtype=torch.uint8, device="cuda")
+    Z = torch.full((M, r), float("nan"), dtype=torch.bfloat16, device="cuda") if r > 0 else None
+    B.quantize_act_lowrank_down_t(fmt, Xd, lam_d, gx, L1d, codes, scales, Z)
+    check_device_error()
+    sc = scales.cpu().numpy()
+    return {
+        "codes": unpack_codes(codes.cpu().numpy(), M, K),
+        "scales": scales_canonical(fmt, sc, M, K),
+        "scale_padding": scales_padding(fmt, sc, M, K),
+        "Z": host_bf16(Z) if r > 0 else np.zeros((M, 0), np.float32),
+        "dev": {"codes": codes, "scales": scales, "Z": Z},
+    }
+
+
+def encode_scales(fmt, scale_bits: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Canonical scale bits [rows][G] -> library buffer bytes (padding rows zero)."""
+    rp = (rows + 127) // 128 * 128
+    if fmt == "nvfp4":
+        buf = np.zeros(rp * K // 16, np.uint8)
+        buf[nvfp4_scale_offsets(rows, K)] = scale_bits
+        return buf
+    buf = np.zeros((K // 64, rp), np.uint16)
+    buf[:, :rows] = scale_bits.T
+    return buf.view(np.uint8).reshape(-1)
+
+
+def pack_codes_bytes(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8).reshape(-1)
+
+
+def run_gemm(fmt, M, N, K, rank, a_codes, a_scales, gx, w_codes, w_scales, gw, Z, L2s, bias):
+    """All operand arguments are host NumPy buffers in library layout (or device tensors)."""
+    def d(x):
+        if x is None:
+            return None
+        if isinstance(x, torch.Tensor):
+            return x
+        return torch.from_numpy(np.ascontiguousarray(x)).cuda()
+    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    B.w4a4_gemm_lowrank_up_t(fmt, M, N, K, rank, d(a_codes), d(a_scales), gx, d(w_codes), d(w_scales), gw,
+                             None if rank == 0 else (Z if isinstance(Z, torch.Tensor) else dev_bf16(Z)),
+                             None if rank == 0 else (L2s if isinstance(L2s, torch.Tensor) else dev_bf16(L2s)),
+                             None if bias is None else (bias if isinstance(bias, torch.Tensor) else dev_bf16(bias)),
+                             Y)
+    check_device_error()
+    return Y
+
+
+def rel_fro(a, b) -> float:
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))

@@ -1,0 +1,81 @@
+"""Decoders from the library's buffer layouts to canonical arrays.
+
+Written from the layout text of include/svdq.h (index functions), separately
+from the library and from the CPU reference; used only by tests.
+"""
+import numpy as np
+
+
+def unpack_codes(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """[rows][K/2] bytes, element k in the low nibble of byte k/2 when k is even."""
+    b = np.asarray(buf, np.uint8).reshape(rows, K // 2)
+    out = np.empty((rows, K), np.uint8)
+    out[:, 0::2] = b & 0xF
+    out[:, 1::2] = b >> 4
+    return out
+
+
+def pack_codes(codes: np.ndarray) -> np.ndarray:
+    c = np.asarray(codes, np.uint8)
+    return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
+
+
+def nvfp4_scale_offsets(rows: int, K: int) -> np.ndarray:
+    """Byte offset of (row, group) in the 128x4 blocked E4M3 scale layout."""
+    r = np.arange(rows)[:, None]
+    g = np.arange(K // 16)[None, :]
+    return ((r // 128) * (K // 64) + g // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + g % 4
+
+
+def nvfp4_scales_canonical(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    b = np.asarray(buf, np.uint8).reshape(-1)
+    return b[nvfp4_scale_offsets(rows, K)]
+
+
+def nvfp4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """Bytes of the padding rows (rows .. ceil(rows/128)*128 - 1)."""
+    rp = (rows + 127) // 128 * 128
+    if rp == rows:
+        return np.zeros(0, np.uint8)
+    b = np.asarray(buf, np.uint8).reshape(-1)
+    off = nvfp4_scale_offsets(rp, K)[rows:]
+    return b[off]
+
+
+def int4_scales_canonical(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    """fp16 [K/64][Rp] group-major -> uint16 bits [rows][K/64]."""
+    rp = (rows + 127) // 128 * 128
+    b = np.asarray(buf).view(np.uint16).reshape(K // 64, rp)
+    return b[:, :rows].T.copy()
+
+
+def int4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    rp = (rows + 127) // 128 * 128
+    b = np.asarray(buf).view(np.uint16).reshape(K // 64, rp)
+    return b[:, rows:].copy()
+
+
+def scales_canonical(fmt: str, buf, rows: int, K: int) -> np.ndarray:
+    return nvfp4_scales_canonical(buf, rows, K) if fmt == "nvfp4" else int4_scales_canonical(buf, rows, K)
+
+
+def scales_padding(fmt: str, buf, rows: int, K: int) -> np.ndarray:
+    return nvfp4_scales_padding(buf, rows, K) if fmt == "nvfp4" else int4_scales_padding(buf, rows, K)
+
+
+def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:
+    return (np.asarray(bits, np.uint16).astype(np.uint32) << 16).view(np.float32)
+
+
+def f32_to_bf16_bits_exact(x: np.ndarray) -> np.ndarray:
+    """Bits of float32 values that are exact bf16 values (asserts exactness)."""
+    x = np.ascontiguousarray(x, np.float32)
+    u = x.view(np.uint32)
+    assert np.all((u & 0xFFFF) == 0), "value is not a bf16 value"
+    return (u >> 16).astype(np.uint16)
+
+
+def bf16_ulp(x: np.ndarray) -> np.ndarray:
+    a = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(a, 2.0 ** -126)))
+    return np.exp2(e - 7)

@@ -1,0 +1,180 @@
+"""The C ABI on the host: exports, argument checks, and the host pack (no GPU).
+
+svdq_pack_weight runs on the CPU, so its codes and scales are compared bit
+for bit with the CPU reference here.  Device calls are only made with
+invalid arguments, which must be rejected before any launch.
+"""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import oracle as O
+from bit_w4a4_quantized_group_b200 import binding as B
+from bit_w4a4_quantized_group_b200 import build as BUILD
+from bit_w4a4_quantized_group_b200 import inputs as I
+
+from layouts import int4_scales_canonical, nvfp4_scales_canonical, scales_padding, unpack_codes
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    BUILD.build()
+    return B.load()
+
+
+def _header_functions():
+    txt = open(os.path.join(ROOT, "include", "svdq.h"), encoding="utf-8").read()
+    txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+    return sorted(set(re.findall(r"\b(svdq_[a-z0-9_]+)\s*\(", txt)))
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = _header_functions()
+    assert len(names) >= 7
+    for n in names:
+        assert hasattr(lib, n), n
+    assert set(names) == set(B.EXPORTED)
+
+
+def test_buffer_sizes(lib):
+    s = B.svdq_buffer_sizes("nvfp4", 300, 640, 768, 32)
+    assert s.a_codes == 300 * 384 and s.w_codes == 640 * 384
+    assert s.a_scales == 384 * 768 // 16          # rows padded to 384
+    assert s.w_scales == 640 * 768 // 16
+    assert s.z == 300 * 32 * 2 and s.l1 == 32 * 768 * 2 and s.l2 == 640 * 32 * 2
+    assert s.y == 300 * 640 * 2 and s.bias == 640 * 2
+    s = B.svdq_buffer_sizes("int4", 300, 640, 768, 0)
+    assert s.a_scales == 384 * (768 // 64) * 2 and s.z == 0
+
+
+@pytest.mark.parametrize("args", [
+    ("nvfp4", 0, 256, 256, 16),      # M < 1
+    ("nvfp4", 64, 200, 256, 16),     # N % 128
+    ("nvfp4", 64, 256, 192, 16),     # K % 128
+    ("nvfp4", 64, 256, 256, 24),     # rank % 16
+    ("nvfp4", 64, 256, 256, 144),    # rank > 128
+    (7, 64, 256, 256, 16),           # bad format
+])
+def test_buffer_sizes_rejects(lib, args):
+    with pytest.raises(B.SvdqError) as e:
+        B.svdq_buffer_sizes(*args)
+    assert e.value.status == B.SVDQ_ERR_INVALID_ARG
+
+
+def _bufs(n=8):
+    return [np.zeros(1 << 16, np.uint8) for _ in range(n)]
+
+
+def test_device_calls_reject_bad_arguments_without_launch(lib):
+    b = _bufs()
+    p = [x.ctypes.data for x in b]
+    # bad K
+    st = B.svdq_quantize_act_lowrank_down("nvfp4", 64, 200, 16, p[0], None, 1.0, p[1], p[2], p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG and B.svdq_last_launch_count() == 0
+    # NULL X
+    st = B.svdq_quantize_act_lowrank_down("nvfp4", 64, 256, 16, None, None, 1.0, p[1], p[2], p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    # misaligned codes pointer
+    st = B.svdq_quantize_act_lowrank_down("nvfp4", 64, 256, 16, p[0], None, 1.0, p[1], p[2] + 1, p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    # non power-of-two activation scale
+    st = B.svdq_quantize_act_lowrank_down("nvfp4", 64, 256, 16, p[0], None, 3.0, p[1], p[2], p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    # INT4 requires unit tensor scales
+    st = B.svdq_quantize_act_lowrank_down("int4", 64, 256, 16, p[0], None, 2.0, p[1], p[2], p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    # rank > 0 needs Z and L1
+    st = B.svdq_quantize_act_lowrank_down("nvfp4", 64, 256, 16, p[0], None, 1.0, None, p[2], p[3], p[4], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    # GEMM: bad N, missing Y, misaligned bias, non power-of-two weight scale
+    args = dict(a=p[0], sa=p[1], w=p[2], sw=p[3], z=p[4], l2=p[5], bias=p[6], y=p[7])
+    st = B.svdq_w4a4_gemm_lowrank_up("nvfp4", 64, 200, 256, 16, args["a"], args["sa"], 1.0, args["w"],
+                                     args["sw"], 1.0, args["z"], args["l2"], args["bias"], args["y"], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    st = B.svdq_w4a4_gemm_lowrank_up("nvfp4", 64, 256, 256, 16, args["a"], args["sa"], 1.0, args["w"],
+                                     args["sw"], 1.0, args["z"], args["l2"], args["bias"], None, None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    st = B.svdq_w4a4_gemm_lowrank_up("nvfp4", 64, 256, 256, 16, args["a"], args["sa"], 1.0, args["w"],
+                                     args["sw"], 1.0, args["z"], args["l2"], args["bias"] + 2, args["y"], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    st = B.svdq_w4a4_gemm_lowrank_up("nvfp4", 64, 256, 256, 16, args["a"], args["sa"], 1.0, args["w"],
+                                     args["sw"], 0.75, args["z"], args["l2"], args["bias"], args["y"], None)
+    assert st == B.SVDQ_ERR_INVALID_ARG
+    assert B.svdq_last_launch_count() == 0
+
+
+def test_status_strings(lib):
+    assert B.status_name(B.SVDQ_OK) == "ok"
+    assert "timed out" in B.status_name(B.SVDQ_ERR_TIMEOUT)
+
+
+# ----------------------------------------------------------------- host pack parity
+
+def _check_pack(fmt, R_nk, L1_rk, L2_nr, gx):
+    N, K = R_nk.shape
+    got = B.pack_weight_np(fmt, R_nk, L1_rk, L2_nr, gx)
+    ref = O.pack_weight(fmt, R_nk, L1_rk, L2_nr, gx)
+    assert got["w_gscale"] == ref["gscale"]
+    assert np.array_equal(unpack_codes(got["w_codes"], N, K), ref["q"]["codes"])
+    if fmt == "nvfp4":
+        assert np.array_equal(nvfp4_scales_canonical(got["w_scales"], N, K), ref["q"]["scale_bits"])
+    else:
+        assert np.array_equal(int4_scales_canonical(got["w_scales"], N, K), ref["q"]["scale_bits"])
+    assert np.all(scales_padding(fmt, got["w_scales"], N, K) == 0)
+    if L1_rk is not None and L1_rk.shape[0] > 0:
+        l1 = (got["L1_bf16"].astype(np.uint32) << 16).view(np.float32)
+        l2 = (got["L2_bf16"].astype(np.uint32) << 16).view(np.float32)
+        assert np.array_equal(l1, ref["L1_bf16"])
+        assert np.array_equal(l2, ref["L2_scaled"])
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_pack_weight_matches_reference_on_tiny_layer(lib, fmt):
+    layer = I.make_layer(I.TINY)
+    prep = O.prepare_layer(fmt, layer.X, layer.W, 16)
+    _check_pack(fmt, prep["R_nk"], prep["L1_rk"].astype(np.float32), prep["L2_nr"].astype(np.float32),
+                prep["act_gscale"])
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("scale_exp", [-12, -3, 0, 6])
+def test_pack_weight_matches_reference_random(lib, fmt, scale_exp):
+    rng = np.random.default_rng(100 + scale_exp)
+    N, K, r = 256, 384, 32
+    R = (rng.standard_normal((N, K)) * 2.0 ** scale_exp).astype(np.float32)
+    # heavy-tailed entries, exact zeros and a zero group
+    R[rng.random((N, K)) < 0.01] *= 40
+    R[3, :] = 0.0
+    R[5, 64:128] = 0.0
+    L1 = rng.standard_normal((r, K)).astype(np.float32)
+    L2 = (rng.standard_normal((N, r)) * 0.1).astype(np.float32)
+    gx = 2.0 ** -7 if fmt == "nvfp4" else 1.0
+    _check_pack(fmt, R, L1, L2, gx)
+
+
+def test_pack_weight_rank0_and_ties(lib):
+    # values placed exactly on E2M1 / INT4 rounding midpoints after scaling
+    N, K = 128, 128
+    R = np.zeros((N, K), np.float32)
+    R[:, 0] = 6.0
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -2.5, -0.1], np.float32)
+    R[:, 1:1 + len(mids)] = mids
+    _check_pack("nvfp4", R, None, None, 1.0)
+    R2 = np.zeros((N, K), np.float32)
+    R2[:, 0] = 7.0
+    R2[:, 1:6] = [0.5, 1.5, 2.5, -0.5, -3.5]
+    _check_pack("int4", R2, None, None, 1.0)
+
+
+def test_pack_weight_rejects(lib):
+    N, K = 128, 128
+    R = np.zeros((N, K), np.float32)
+    with pytest.raises(B.SvdqError):
+        B.pack_weight_np("nvfp4", R, None, None, 3.0)     # not a power of two
+    with pytest.raises(B.SvdqError):
+        B.pack_weight_np("int4", R, None, None, 0.5)      # INT4 needs g_x = 1

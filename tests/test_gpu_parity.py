@@ -1,0 +1,177 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU reference.
+
+Bars (from the header contract and the reference's readings):
+  * codes and scales: bit exact, including the zero padding rows;
+  * Z: within one bf16 ulp of bf16(fp64 X_hat L1^T), plus the fp32
+    accumulation slack 2^-16 * sum_k |x_hat_k L1_jk|;
+  * Y: relative Frobenius error <= 1e-3 against bf16(Y64), Y64 being the fp64
+    reference on the same quantized operands and the same Z.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from bit_w4a4_quantized_group_b200 import binding as B
+from bit_w4a4_quantized_group_b200 import build as BUILD
+from bit_w4a4_quantized_group_b200 import inputs as I
+
+from gpu_helpers import encode_scales, host_bf16, pack_codes_bytes, rel_fro, run_gemm, run_prologue
+from layouts import bf16_ulp
+
+pytestmark = pytest.mark.gpu
+
+Y_TOL = 1e-3
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    BUILD.build()
+    B.load()
+
+
+def _layer(M, K, N, rank, seed, fmt, outliers=4):
+    cfg = I.LayerConfig(name="t", b=M, m=K, n=N, rank=rank, seed=seed, outlier_count=outliers,
+                        outlier_mult=30.0, spike_rank=4, spike_sigma=1.5)
+    layer = I.make_layer(cfg)
+    prep = O.prepare_layer(fmt, layer.X, layer.W, rank)
+    return layer, prep
+
+
+def _check_z(Zg, xh, L1_rk, Zref):
+    if L1_rk is None or L1_rk.shape[0] == 0:
+        return
+    S = np.abs(xh.astype(np.float64)) @ np.abs(L1_rk.astype(np.float64)).T
+    err = np.abs(Zg.astype(np.float64) - Zref.astype(np.float64))
+    tol = bf16_ulp(Zref) + 2.0 ** -16 * S
+    assert np.all(err <= tol), f"Z max excess {np.max(err - tol)}"
+    # most elements round identically
+    assert np.mean(Zg == Zref) > 0.99
+
+
+def _check_prologue(fmt, X, lam, gx, L1_rk):
+    got = run_prologue(fmt, X, lam, gx, L1_rk)
+    ref = O.prologue(fmt, X, lam, gx, L1_rk)
+    np.testing.assert_array_equal(got["codes"], ref["q"]["codes"])
+    np.testing.assert_array_equal(got["scales"], ref["q"]["scale_bits"])
+    assert np.all(got["scale_padding"] == 0)
+    _check_z(got["Z"], ref["xhat"], L1_rk, ref["Z"])
+    return got, ref
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
+                                      (96, 512, 128)])
+def test_prologue_parity(fmt, M, K, rank):
+    layer, prep = _layer(M, K, 256, rank, seed=7 + M + rank, fmt=fmt)
+    _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_prologue_without_smoothing_and_zero_rows(fmt):
+    rng = np.random.default_rng(5)
+    X = I.to_bf16(rng.standard_normal((200, 384)) * 3)
+    X[7] = 0.0                      # an all-zero row: zero scales, zero codes
+    X[9, 64:128] = 0.0              # a zero group
+    gx = O.pow2_global_scale(np.abs(X).max()) if fmt == "nvfp4" else 1.0
+    L1 = I.to_bf16(rng.standard_normal((16, 384)) * 0.05).astype(np.float64)
+    _check_prologue(fmt, X, None, gx, L1)
+
+
+def test_prologue_rounding_ties_nvfp4():
+    """Values on E2M1 rounding midpoints (scale exactly 1) and small negatives (-0 code)."""
+    M, K = 128, 128
+    X = np.zeros((M, K), np.float32)
+    X[:, 0] = 6.0
+    vals = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25, -0.75, -2.5, -5.0, -0.125, 0.125,
+                     -0.0078125, 4.5], np.float32)
+    X[:, 1:16] = vals
+    X[:, 16] = -6.0
+    X[:, 17:32] = -vals
+    X = I.to_bf16(X)
+    got, ref = _check_prologue("nvfp4", X, None, 1.0, None)
+    assert got["codes"][0, 1] == 0 and got["codes"][0, 2] == 2 and got["codes"][0, 8] == 8
+
+
+def test_prologue_rounding_ties_int4():
+    M, K = 128, 128
+    X = np.zeros((M, K), np.float32)
+    X[:, 0] = 7.0
+    X[:, 1:9] = [0.5, 1.5, 2.5, 3.5, -0.5, -1.5, -2.5, -6.5]
+    X = I.to_bf16(X)
+    _check_prologue("int4", X, None, 1.0, None)
+
+
+def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
+    layer, prep = _layer(M, K, N, rank, seed=seed, fmt=fmt)
+    gx = prep["act_gscale"]
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
+    pro = O.prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"] if rank else None)
+    bias = layer.bias if with_bias else None
+    ref = O.gemm_forward(pro["q"], gx, packed["q"], packed["gscale"], pro["Z"], packed["L2_bf16"], bias)
+    Y = run_gemm(fmt, M, N, K, rank,
+                 pack_codes_bytes(pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
+                 pack_codes_bytes(packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
+                 packed["gscale"], pro["Z"], packed["L2_scaled"], bias)
+    Yg = host_bf16(Y)
+    assert np.all(np.isfinite(Yg))
+    e_ref = rel_fro(Yg, ref["Y"])
+    e_64 = rel_fro(Yg, ref["Y64"])
+    assert e_ref <= Y_TOL, (e_ref, e_64)
+    assert e_64 <= 4e-3
+    return Yg, ref
+
+
+@pytest.mark.parametrize("M,N,K,rank", [(300, 640, 640, 32), (256, 512, 512, 16), (128, 256, 256, 0),
+                                        (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64)])
+def test_gemm_parity_nvfp4(M, N, K, rank):
+    _gemm_case("nvfp4", M, N, K, rank, seed=11 + M + N + rank)
+
+
+def test_gemm_parity_nvfp4_no_bias():
+    _gemm_case("nvfp4", 160, 512, 512, 32, seed=3, with_bias=False)
+
+
+def test_gemm_lowrank_branch_is_added_nvfp4():
+    """Y(r) - Y(r=0 on the same 4-bit operands) equals Z L2 (the branch really lands in Y)."""
+    fmt, M, N, K, rank = "nvfp4", 128, 256, 256, 32
+    layer, prep = _layer(M, K, N, rank, seed=19, fmt=fmt)
+    gx = prep["act_gscale"]
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
+    pro = O.prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"])
+    args = (pack_codes_bytes(pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
+            pack_codes_bytes(packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
+            packed["gscale"])
+    Y1 = host_bf16(run_gemm(fmt, M, N, K, rank, *args, pro["Z"], packed["L2_scaled"], None)).astype(np.float64)
+    Y0 = host_bf16(run_gemm(fmt, M, N, K, 0, *args, None, None, None)).astype(np.float64)
+    branch = pro["Z"].astype(np.float64) @ packed["L2_bf16"].astype(np.float64).T
+    assert rel_fro(Y1 - Y0, branch) < 2e-2
+
+
+@pytest.mark.parametrize("fmt,rank", [("nvfp4", 32), ("nvfp4", 0), ("nvfp4", 128)])
+def test_layer_end_to_end_small(fmt, rank):
+    """Prologue then GEMM on the device (Z never leaves the GPU) vs the reference layer."""
+    M, K, N = 384, 768, 768
+    layer, prep = _layer(M, K, N, rank, seed=23 + rank, fmt=fmt)
+    gx = prep["act_gscale"]
+    pk = B.pack_weight_np(fmt, prep["R_nk"].astype(np.float32), prep["L1_rk"].astype(np.float32) if rank else None,
+                          prep["L2_nr"].astype(np.float32) if rank else None, gx)
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
+    L1 = packed["L1_bf16"] if rank else None
+    got = run_prologue(fmt, layer.X, prep["lam"], gx, L1)
+    L2s_dev = None
+    if rank:
+        L2s_dev = torch.from_numpy(pk["L2_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    Y = run_gemm(fmt, M, N, K, rank, got["dev"]["codes"], got["dev"]["scales"], gx,
+                 pk["w_codes"], pk["w_scales"], pk["w_gscale"], got["dev"]["Z"], L2s_dev, layer.bias)
+    ref = O.layer_forward(fmt, layer.X, prep["lam"], gx, packed, layer.bias)
+    Yg = host_bf16(Y)
+    # the GPU Z may differ from the reference Z by one bf16 ulp; Y is compared with the
+    # reference computed on the GPU's Z so that the bar isolates the GEMM
+    ref_gz = O.gemm_forward(ref["q"], gx, packed["q"], packed["gscale"], got["Z"], packed["L2_bf16"], layer.bias)
+    assert rel_fro(Yg, ref_gz["Y"]) <= Y_TOL
+    assert rel_fro(Yg, ref["Y"]) <= 2e-3
+    # and the layer approximates the unquantized X W + b
+    exact = layer.X.astype(np.float64) @ layer.W + layer.bias.astype(np.float64)
+    assert rel_fro(Yg, exact) < 0.15

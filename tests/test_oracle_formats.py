@@ -246,3 +246,12 @@ def test_planted_round_half_up_is_caught():
     """Rounding half away from zero (instead of to even) breaks the argmin pin on ties."""
     t = np.array([0.5, 1.5, 2.5, -2.5], np.float64)
     assert not np.array_equal(np.floor(t + 0.5), np.rint(t))
+
+
+def test_pow2_global_scale_boundaries():
+    # amax exactly 6 * 448 * 2**e must give g = 2**e (amax / (6 g) == 448 is allowed)
+    for e in (-12, -3, 0, 5):
+        amax = 6 * 448 * 2.0 ** e
+        assert O.pow2_global_scale(amax) == 2.0 ** e
+        assert O.pow2_global_scale(np.nextafter(amax, 1e30)) == 2.0 ** (e + 1)
+        assert O.pow2_global_scale(np.nextafter(amax, 0)) == 2.0 ** e
