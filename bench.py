@@ -1,0 +1,397 @@
+#!/usr/bin/env python
+"""Benchmark of the W4A4 + low-rank linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl svdq|reference]
+                    [--workload mlp_up|qkv|mlp_down|tiny] [--format nvfp4|int4] [--rank R]
+
+One step = the whole hot path on one batch: the prologue (smooth, quantize,
+down-project) and the fused W4A4 GEMM (+ up-projection + bias), i.e. one
+forward of the DiT MLP-up layer 4608 x 3072 x 12288, rank 32, NVFP4 by
+default.  Inputs are seeded synthetic data (bit_w4a4_quantized_group_b200/inputs.py);
+weights are
+decomposed offline (not timed).  Each timed step is bracketed by CUDA events
+on the launching stream; a 512 MB write between steps flushes the 126 MB L2
+outside the events.  Multi-GPU runs (torchrun) are independent replicas, one
+layer per GPU (weak scaling); time is the max over ranks.
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4+low-rank linear effective TFLOPS"
+UNIT = "TFLOP/s"
+FALLBACK_BF16_TFLOPS = 1590.0
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
+    ap.add_argument("--workload", default="mlp_up")
+    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "int4"])
+    ap.add_argument("--rank", type=int, default=None)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), float(d.get("bf16_tflops_sustained", d["bf16_tflops"])), \
+            float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_BF16_TFLOPS, 1400.0, FALLBACK_HBM_GBS, "fallback"
+
+
+def workload(args):
+    from bit_w4a4_quantized_group_b200 import inputs as I
+    cfg = I.NAMED[args.workload]
+    if args.rank is not None and args.rank != cfg.rank:
+        import dataclasses
+        cfg = dataclasses.replace(cfg, rank=args.rank)
+    return cfg
+
+
+def prepare_layer(cfg, fmt, device):
+    from bit_w4a4_quantized_group_b200 import inputs as I
+    from bit_w4a4_quantized_group_b200 import prepare as P
+    layer = I.make_layer(cfg)
+    prep = P.prepare(fmt, layer.X, layer.W, cfg.rank, device=device)
+    packed = P.pack(fmt, prep)
+    return layer, prep, packed
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        try:
+            with open(self.path) as f:
+                for line in f:
+                    parts = [p.strip() for p in line.split(",")]
+                    if len(parts) >= 9:
+                        rows.append(parts)
+            os.unlink(self.path)
+        except Exception:
+            return None
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
+        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def source_hash(path):
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
+def recorded_traffic(kernel_src, workload_name):
+    """DRAM bytes per launch from a committed ncu summary, only if the kernel source is unchanged."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        e = d[workload_name]
+        if e["source_sha256_16"] != source_hash(kernel_src):
+            return None
+        return float(e["dram_bytes_per_launch"])
+    except Exception:
+        return None
+
+
+# ----------------------------------------------------------------------------- CPU reference timing
+
+def time_oracle(cfg, fmt, prep, X, budget_s=15.0, min_rows=16, max_rows=256):
+    """The CPU reference forward (prologue + GEMM, fp64) on a sample of rows."""
+    import oracle as O
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], prep["act_gscale"])
+    rows = min_rows
+    t0 = time.perf_counter()
+    O.layer_forward(fmt, X[:rows], prep["lam"], prep["act_gscale"], packed, None)
+    dt = time.perf_counter() - t0
+    # grow the sample towards ~budget_s of CPU work
+    while dt * 2 < budget_s and rows * 2 <= max_rows:
+        rows *= 2
+        t0 = time.perf_counter()
+        O.layer_forward(fmt, X[:rows], prep["lam"], prep["act_gscale"], packed, None)
+        dt = time.perf_counter() - t0
+    tflops = 2.0 * rows * cfg.n * cfg.m / dt / 1e12
+    return {"value": tflops, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{rows} of {cfg.b} rows of {cfg.name} ({fmt}, r={cfg.rank}); prologue + GEMM in fp64 "
+                      f"NumPy, {dt:.2f} s"}, packed
+
+
+def run_reference(args):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    cfg = workload(args)
+    from bit_w4a4_quantized_group_b200 import inputs as I
+    import oracle as O
+    layer = I.make_layer(cfg)
+    prep = O.prepare_layer(args.format, layer.X, layer.W, cfg.rank)
+    prep = {"lam": prep["lam"], "R_nk": prep["R_nk"], "L1_rk": prep["L1_rk"], "L2_nr": prep["L2_nr"],
+            "act_gscale": prep["act_gscale"]}
+    packed = O.pack_weight(args.format, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], prep["act_gscale"])
+    rows = 16
+    for _ in range(args.warmup):
+        O.layer_forward(args.format, layer.X[:rows], prep["lam"], prep["act_gscale"], packed, None)
+    times = []
+    for i in range(args.steps):
+        lo = (i * rows) % cfg.b
+        t0 = time.perf_counter()
+        O.layer_forward(args.format, layer.X[lo:lo + rows], prep["lam"], prep["act_gscale"], packed, None)
+        times.append(time.perf_counter() - t0)
+    t = sum(times) / len(times)
+    value = 2.0 * rows * cfg.n * cfg.m / t / 1e12
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+    except Exception:
+        cores = os.cpu_count() or 1
+    out = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_dict(cfg, args.format, "host memory (CPU reference)"),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": f"{rows} rows of {cfg.b} per step ({cfg.name}, {args.format}, r={cfg.rank})"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(out))
+    return 0
+
+
+def config_dict(cfg, fmt, l2):
+    return {"workload": f"{cfg.name} {cfg.b}x{cfg.m}x{cfg.n} r={cfg.rank} {fmt}", "M": cfg.b, "K": cfg.m,
+            "N": cfg.n, "rank": cfg.rank, "format": fmt, "bias": cfg.with_bias, "l2": l2}
+
+
+# ----------------------------------------------------------------------------- GPU path
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if not torch.cuda.is_available():
+        raise RuntimeError("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300), device_id=device)
+
+    from bit_w4a4_quantized_group_b200 import binding as B
+    from bit_w4a4_quantized_group_b200 import build as BUILD
+    from bit_w4a4_quantized_group_b200.layer import W4A4LowRankLinear
+    BUILD.build()
+    B.load()
+
+    cfg = workload(args)
+    fmt = args.format
+    layer, prep, packed = prepare_layer(cfg, fmt, str(device))
+    M, K, N, r = cfg.b, cfg.m, cfg.n, cfg.rank
+    lin = W4A4LowRankLinear(fmt, N, K, packed, prep["lam"], prep["act_gscale"], layer.bias, device=device)
+    from bit_w4a4_quantized_group_b200.inputs import bf16_bits
+    X = torch.from_numpy(bf16_bits(layer.X).view(np.int16)).to(device).view(torch.bfloat16)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+
+    # warm-up (untimed)
+    for _ in range(args.warmup):
+        flush.zero_()
+        lin.forward(X, Y)
+    barrier()
+    st, site = B.svdq_get_last_device_error(None)
+    if st != B.SVDQ_OK:
+        raise RuntimeError(f"device error {st} at site {site}")
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    launches = 0
+    barrier()
+    for i in range(args.steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        lin.prologue_only(X)
+        launches += B.svdq_last_launch_count()
+        ev[i][1].record(stream)
+        lin.gemm_only(M, Y)
+        launches += B.svdq_last_launch_count()
+        ev[i][2].record(stream)
+    barrier()
+    clk = clocks.stop()
+    t_pro = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps * 1e-3
+    t_gemm = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps * 1e-3
+    t_step = t_pro + t_gemm
+
+    # low-rank overhead: the same GEMM without the branch (not part of the headline)
+    gemm0 = []
+    for i in range(max(5, args.steps // 2)):
+        flush.zero_()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lin.gemm_only(M, Y, rank=0)
+        b.record(stream)
+        gemm0.append((a, b))
+    torch.cuda.synchronize()
+    t_gemm0 = sum(a.elapsed_time(b) for a, b in gemm0) / len(gemm0) * 1e-3
+    lin.forward(X, Y)                        # restore Y with the branch
+    st, site = B.svdq_get_last_device_error(None)
+    if st != B.SVDQ_OK:
+        raise RuntimeError(f"device error {st} at site {site}")
+
+    # end to end through the public layer API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        Xh = torch.empty((M, K), dtype=torch.bfloat16, pin_memory=True)
+        Xh.copy_(X.cpu())
+        Yh = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+        for _ in range(2):
+            X.copy_(Xh, non_blocking=True)
+            lin.forward(X, Y)
+            Yh.copy_(Y, non_blocking=True)
+        barrier()
+        ee = []
+        for i in range(args.steps):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            X.copy_(Xh, non_blocking=True)
+            lin.forward(X, Y)
+            Yh.copy_(Y, non_blocking=True)
+            b.record(stream)
+            ee.append((a, b))
+        barrier()
+        t_e2e = sum(a.elapsed_time(b) for a, b in ee) / len(ee) * 1e-3
+        e2e = {"t": t_e2e, "h2d": M * K * 2, "d2h": M * N * 2}
+
+    # max over ranks
+    vals = torch.tensor([t_step, t_pro, t_gemm, t_gemm0, e2e["t"] if e2e else 0.0], dtype=torch.float64,
+                        device=device)
+    if world > 1:
+        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
+    t_step, t_pro, t_gemm, t_gemm0, t_e2e = vals.tolist()
+
+    flops = 2.0 * M * N * K
+    value = world * flops / t_step / 1e12
+    bf16_burst, bf16_sus, hbm, peak_src = peaks()
+    if fmt == "nvfp4":
+        peak = bf16_burst * 4.0              # dense FP4 = 4 x dense bf16 (nominal ratio 9 : 2.25)
+        peak_note = f"dense FP4 = 4 x {peak_src} bf16 burst"
+        src = os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc", "gemm_nvfp4.cu")
+    else:
+        peak = bf16_burst * 2.0              # dense INT8 = 2 x dense bf16 (nominal ratio 4.5 : 2.25)
+        peak_note = f"dense INT8 = 2 x {peak_src} bf16 burst"
+        src = os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc", "gemm_int4.cu")
+    alg_flops = flops + 2.0 * M * N * r
+    achieved = alg_flops / t_gemm / 1e12
+    traffic = recorded_traffic(src, f"{cfg.name}_{fmt}_r{r}")
+    g = 16 if fmt == "nvfp4" else 64
+    sf = 1 if fmt == "nvfp4" else 2
+    pro_bytes = 2 * M * K + M * K / 2 + M * K / g * sf + 2 * M * r + 2 * r * K + (4 * K)
+    out = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": fmt, "data": "synthetic",
+        "config": config_dict(cfg, fmt, "flushed: 512 MB write between timed steps, outside the events"),
+        "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": traffic, "kernel": f"gemm_{fmt}",
+                     "peak_source": peak_note},
+        "gemm_us": t_gemm * 1e6, "prologue_us": t_pro * 1e6, "gemm_r0_us": t_gemm0 * 1e6,
+        "lowrank_overhead_pct": 100.0 * (t_gemm / t_gemm0 - 1.0),
+        "gemm_frac_fp4_peak": (flops / t_gemm / 1e12) / peak,
+        "prologue": {"bound": "hbm", "GB/s": pro_bytes / t_pro / 1e9, "peak": hbm,
+                     "frac": pro_bytes / t_pro / 1e9 / hbm, "bytes": pro_bytes},
+        "gpu_launches": launches,
+        "clocks": clk,
+    }
+    if e2e:
+        out["e2e"] = {"value": world * flops / t_e2e / 1e12, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+                      "d2h_bytes_per_step": e2e["d2h"]}
+    if world == 1 and rank == 0 and not args.no_cpu_baseline:
+        cb, _ = time_oracle(cfg, fmt, prep, layer.X)
+        out["cpu_baseline"] = cb
+    if rank == 0:
+        print(json.dumps(out))
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

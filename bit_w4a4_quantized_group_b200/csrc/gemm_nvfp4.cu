@@ -1,23 +1,28 @@
-// NVFP4 W4A4 GEMM with the fused low-rank up projection (sm_100a).
+// NVFP4 W4A4 GEMM with the fused low-rank up projection (sm_100a, CTA pairs).
 //
 // "SVDQuant 阅读笔记：用少量高精度计算保护 4-bit 扩散模型", §6.1 "算法 2"
 // steps 4-8 and eq.(7): the 4-bit product Q(X_hat) Q(R) and the 16-bit branch
 // Z L2 are merged before the single write of Y.
 //
 // B200 design:
-//   * persistent CTAs (one per SM), 128 x 256 output tiles, K staged 256
-//     E2M1 elements (128 bytes per row) at a time through a 4-deep TMA ring;
-//   * warp 0 issues TMA (codes as 128B-swizzled tiles, E4M3 scale blocks as
-//     plain bulk copies), warp 1 issues tcgen05 block-scaled MMAs
-//     (kind::mxf4nvf4, UE4M3 scales per 16 elements) into an fp32 TMEM
-//     accumulator, after moving the scale blocks smem -> TMEM with tcgen05.cp;
-//   * the low-rank branch is ceil(r/64) extra pipeline steps in which the ring
-//     slots hold Z (bf16, [128 x 64]) and L2s (bf16, [256 x 64]); warp 1 adds
-//     Z L2s^T into the *same* accumulator with kind::f16 MMAs.  L2s was divided
-//     by (g_x g_w) at pack time, so one multiply by g_x g_w in the epilogue
-//     scales both terms correctly and Y gets no extra pass;
-//   * warps 2-9 drain TMEM (tcgen05.ld), free it for the next tile at once,
-//     then apply g_x g_w and the bias and store bf16 Y.
+//   * clusters of two CTAs on neighbouring SMs compute 256 x 256 output tiles
+//     with tcgen05 cta_group::2 MMAs (M = 256: each CTA holds 128 rows of A and
+//     128 rows of B; the pair's tensor cores share the B halves, which halves
+//     the shared-memory operand traffic per SM against a one-CTA 128 x 256 tile);
+//   * persistent clusters walk the tile list; K is staged 256 E2M1 elements
+//     (128 bytes per row) at a time through a 5-deep TMA ring per CTA.  Every
+//     load is a TMA tile load into the issuing CTA's own shared memory whose
+//     completion is counted on the leader CTA's barrier (no multicast loads);
+//   * block scales (E4M3, one per 16 elements) are TMA-loaded as 512-byte
+//     "128 rows x 4 groups" blocks and moved to TMEM with tcgen05.cp; each CTA
+//     holds its 128 rows of A-scales and all 256 columns of B-scales;
+//   * the leader's MMA warp issues kind::mxf4nvf4 block-scaled MMAs into an fp32
+//     TMEM accumulator and then ceil(r/64) extra pipeline steps in which the
+//     ring slots hold Z (bf16) and L2s (bf16): kind::f16 MMAs add Z L2s^T into the
+//     *same* accumulator.  L2s was divided by (g_x g_w) at pack time, so the
+//     epilogue's single multiply by g_x g_w scales both terms and Y is written once;
+//   * eight epilogue warps per CTA drain TMEM (tcgen05.ld), release it to the
+//     MMA warp at once, then apply g_x g_w and the bias and store bf16 Y.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -28,25 +33,33 @@
 namespace svdq {
 namespace {
 
-constexpr int kBM = 128, kBN = 256;
+constexpr int kBM = 256, kBN = 256;           // pair tile
+constexpr int kRows = 128;                    // A rows (and B rows) per CTA
 constexpr int kKTile = 256;                   // E2M1 elements per pipeline step
-constexpr int kStages = 4;
+constexpr int kStages = 5;
 constexpr int kThreads = 320;                 // producer, MMA, 8 epilogue warps
-constexpr uint32_t kABytes = kBM * 128;       // 16 KB
-constexpr uint32_t kBBytes = kBN * 128;       // 32 KB
+constexpr int kEpiWarps = 8;
+constexpr uint32_t kABytes = kRows * 128;     // 16 KB
+constexpr uint32_t kBBytes = kRows * 128;     // 16 KB
+constexpr uint32_t kSfaBytes = 2048;          // 128 rows x 16 groups
+constexpr uint32_t kSfbBytes = 4096;          // 256 rows x 16 groups
 constexpr uint32_t kSfaOff = kABytes + kBBytes;
-constexpr uint32_t kSfbOff = kSfaOff + 2048;
-constexpr uint32_t kStageBytes = kSfbOff + 4096;   // 54 KB
+constexpr uint32_t kSfbOff = kSfaOff + kSfaBytes;
+constexpr uint32_t kStageBytes = kSfbOff + kSfbBytes;   // 38 KB
+constexpr uint32_t kTxMain = 2 * kStageBytes;            // both CTAs
+constexpr uint32_t kTxLowRank = 2 * (kABytes + kBBytes);
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSfa = 256, kTmemSfb = 272;
 
-__host__ __device__ constexpr uint32_t idesc_nvf4(int n) {
+__host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
+  // E2M1 x E2M1, UE4M3 scales, K-major A and B, dense
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (0u << 23) |
-         (static_cast<uint32_t>(kBM >> 4) << 24);
+         (static_cast<uint32_t>(m >> 4) << 24);
 }
-__host__ __device__ constexpr uint32_t idesc_bf16(int n) {
+__host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
+  // bf16 x bf16 -> fp32, K-major A and B
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
-         (static_cast<uint32_t>(kBM >> 4) << 24);
+         (static_cast<uint32_t>(m >> 4) << 24);
 }
 
 struct SharedTail {
@@ -60,6 +73,7 @@ struct SharedTail {
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+                      const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_z, const __grid_constant__ CUtensorMap tmap_l2,
                       GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -69,6 +83,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();      // 0 = leader of the pair
+  const int cluster = blockIdx.x >> 1;
+  const int nclusters = gridDim.x >> 1;
   const int nk_main = (p.K + kKTile - 1) / kKTile;
   const int nk_lr = (p.rank + 63) / 64;
   const int nk = nk_main + nk_lr;
@@ -80,124 +97,118 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&sh->empty[s], 1);
     }
     ptx::mbar_init(&sh->acc_full, 1);
-    ptx::mbar_init(&sh->acc_empty, 8);
+    ptx::mbar_init(&sh->acc_empty, 2 * kEpiWarps);
     sh->abort_flag = 0;
     ptx::fence_mbar_init();
   }
   if (warp == 1) {
-    ptx::tmem_alloc(&sh->tmem_base, kTmemCols);
-    ptx::tmem_relinquish();
+    ptx::tmem_alloc_pair(&sh->tmem_base, kTmemCols);
+    ptx::tmem_relinquish_pair();
   }
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
 
   if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ TMA producer (both CTAs)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmap_a);
       ptx::prefetch_tmap(&tmap_b);
+      ptx::prefetch_tmap(&tmap_sfa);
+      ptx::prefetch_tmap(&tmap_sfb);
       if (nk_lr > 0) {
         ptx::prefetch_tmap(&tmap_z);
         ptx::prefetch_tmap(&tmap_l2);
       }
       int it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
         const int mb = t % p.tiles_m, nb = t / p.tiles_m;
-        const int m0 = mb * kBM, n0 = nb * kBN;
-        const bool full_n = (n0 + kBN) <= p.N;
+        const int m0 = mb * kBM + static_cast<int>(rank) * kRows;     // this CTA's A rows
+        const int n0 = nb * kBN;
+        const int nb0 = n0 + static_cast<int>(rank) * kRows;          // this CTA's B rows
         for (int k = 0; k < nk; ++k, ++it) {
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!wait_bounded(&sh->empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteGemmEmpty)) { ok = false; break; }
-          uint8_t* st = smem + s * kStageBytes;
+          const uint32_t full_leader = ptx::mapa_shared(ptx::smem_u32(&sh->full[s]), 0);
+          const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
           if (k < nk_main) {
-            const int kb0 = k * (kKTile / 64);                 // first 64-element block
-            const int nkb = min(kKTile / 64, kblk64 - kb0);
-            const uint32_t sfbytes = nkb * 512u;
-            const uint32_t bytes = kABytes + kBBytes + sfbytes * (full_n ? 3u : 2u);
-            ptx::mbar_arrive_expect_tx(&sh->full[s], bytes);
-            ptx::tma_load_2d(st, &tmap_a, &sh->full[s], k * (kKTile / 2), m0);
-            ptx::tma_load_2d(st + kABytes, &tmap_b, &sh->full[s], k * (kKTile / 2), n0);
-            ptx::bulk_load(st + kSfaOff, p.a_scales + (static_cast<size_t>(mb) * kblk64 + kb0) * 512, sfbytes,
-                           &sh->full[s]);
-            ptx::bulk_load(st + kSfbOff, p.w_scales + (static_cast<size_t>(n0 / 128) * kblk64 + kb0) * 512,
-                           sfbytes, &sh->full[s]);
-            if (full_n)
-              ptx::bulk_load(st + kSfbOff + 2048,
-                             p.w_scales + (static_cast<size_t>(n0 / 128 + 1) * kblk64 + kb0) * 512, sfbytes,
-                             &sh->full[s]);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], kTxMain);
+            ptx::tma_load_2d_pair(st, &tmap_a, full_leader, k * (kKTile / 2), m0);
+            ptx::tma_load_2d_pair(st + kABytes, &tmap_b, full_leader, k * (kKTile / 2), nb0);
+            ptx::tma_load_3d_pair(st + kSfaOff, &tmap_sfa, full_leader, 0, k * (kKTile / 64), m0 / 128);
+            ptx::tma_load_3d_pair(st + kSfbOff, &tmap_sfb, full_leader, 0, k * (kKTile / 64), n0 / 128);
           } else {
             const int c = k - nk_main;
-            ptx::mbar_arrive_expect_tx(&sh->full[s], kABytes + kBBytes);
-            ptx::tma_load_2d(st, &tmap_z, &sh->full[s], c * 64, m0);
-            ptx::tma_load_2d(st + kABytes, &tmap_l2, &sh->full[s], c * 64, n0);
+            if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], kTxLowRank);
+            ptx::tma_load_2d_pair(st, &tmap_z, full_leader, c * 64, m0);
+            ptx::tma_load_2d_pair(st + kABytes, &tmap_l2, full_leader, c * 64, nb0);
           }
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    int it = 0;
-    uint32_t acc_ph = 0;
-    bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-      const int n0 = (t / p.tiles_m) * kBN;
-      const int ntile = min(kBN, p.N - n0);
-      const uint32_t id4 = idesc_nvf4(ntile);
-      const uint32_t id16 = idesc_bf16(ntile);
-      if (!wait_bounded(&sh->acc_empty, acc_ph ^ 1u, abort_flag, p.err, kErrSiteGemmAccEmpty)) break;
-      ptx::tc_fence_after();
-      for (int k = 0; k < nk; ++k, ++it) {
-        const int s = it % kStages;
-        const uint32_t ph = (it / kStages) & 1;
-        if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull)) { ok = false; break; }
+    // ------------------------------------------------------------ MMA issuer (leader CTA only)
+    if (rank == 0) {
+      int it = 0;
+      uint32_t acc_ph = 0;
+      bool ok = true;
+      const uint32_t id4 = idesc_nvf4(kBM, kBN);
+      const uint32_t id16 = idesc_bf16(kBM, kBN);
+      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
+        if (!wait_bounded(&sh->acc_empty, acc_ph ^ 1u, abort_flag, p.err, kErrSiteGemmAccEmpty)) break;
         ptx::tc_fence_after();
-        if (lane == 0) {
-          const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
-          if (k < nk_main) {
-            const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
-            for (int kb = 0; kb < nkb; ++kb) {
-              ptx::tmem_cp_32x128b_warpx4(tmem + kTmemSfa + kb * 4, ptx::sdesc_sf(st + kSfaOff + kb * 512));
-              ptx::tmem_cp_32x128b_warpx4(tmem + kTmemSfb + kb * 8, ptx::sdesc_sf(st + kSfbOff + kb * 512));
-              if (ntile == kBN)
-                ptx::tmem_cp_32x128b_warpx4(tmem + kTmemSfb + kb * 8 + 4,
-                                            ptx::sdesc_sf(st + kSfbOff + 2048 + kb * 512));
+        for (int k = 0; k < nk; ++k, ++it) {
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull)) { ok = false; break; }
+          ptx::tc_fence_after();
+          if (lane == 0) {
+            const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
+            if (k < nk_main) {
+              const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
+              for (int kb = 0; kb < nkb; ++kb) {
+                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfa + kb * 4, ptx::sdesc_sf(st + kSfaOff + kb * 512));
+                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfb + kb * 8, ptx::sdesc_sf(st + kSfbOff + kb * 512));
+                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfb + kb * 8 + 4,
+                                                 ptx::sdesc_sf(st + kSfbOff + 2048 + kb * 512));
+              }
+              for (int kb = 0; kb < nkb; ++kb) {
+                ptx::umma_nvf4_pair(tmem, ptx::sdesc_sw128(st + kb * 32), ptx::sdesc_sw128(st + kABytes + kb * 32),
+                                    id4, tmem + kTmemSfa + kb * 4, tmem + kTmemSfb + kb * 8,
+                                    (k | kb) != 0 ? 1u : 0u);
+              }
+            } else {
+              const int c = k - nk_main;
+              const int nmma = min(64, p.rank - c * 64) / 16;
+              for (int j = 0; j < nmma; ++j)
+                ptx::umma_f16_pair(tmem, ptx::sdesc_sw128(st + j * 32), ptx::sdesc_sw128(st + kABytes + j * 32),
+                                   id16, 1u);
             }
-            for (int kb = 0; kb < nkb; ++kb) {
-              ptx::umma_nvf4(tmem, ptx::sdesc_sw128(st + kb * 32), ptx::sdesc_sw128(st + kABytes + kb * 32), id4,
-                             tmem + kTmemSfa + kb * 4, tmem + kTmemSfb + kb * 8, (k | kb) != 0 ? 1u : 0u);
-            }
-          } else {
-            const int c = k - nk_main;
-            const int nmma = min(64, p.rank - c * 64) / 16;
-            for (int j = 0; j < nmma; ++j) {
-              ptx::umma_f16(tmem, ptx::sdesc_sw128(st + j * 32), ptx::sdesc_sw128(st + kABytes + j * 32), id16,
-                            1u);
-            }
+            ptx::tc_commit_pair(&sh->empty[s], 0x3);
           }
-          ptx::tc_commit(&sh->empty[s]);
+          __syncwarp();
         }
+        if (!ok) break;
+        if (lane == 0) ptx::tc_commit_pair(&sh->acc_full, 0x3);
         __syncwarp();
+        acc_ph ^= 1u;
       }
-      if (!ok) break;
-      if (lane == 0) ptx::tc_commit(&sh->acc_full);
-      __syncwarp();
-      acc_ph ^= 1u;
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9)
+    // ------------------------------------------------------------ epilogue (warps 2-9, both CTAs)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int h = (warp - 2) >> 2;          // column half of the 256-wide tile
+    const uint32_t acc_empty_leader = ptx::mapa_shared(ptx::smem_u32(&sh->acc_empty), 0);
     uint32_t acc_ph = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    for (int t = cluster; t < p.num_tiles; t += nclusters) {
       const int mb = t % p.tiles_m, nb = t / p.tiles_m;
-      const int m0 = mb * kBM, n0 = nb * kBN;
-      const int ntile = min(kBN, p.N - n0);
-      const bool active = (h * 128) < ntile;
+      const int m0 = mb * kBM + static_cast<int>(rank) * kRows;
+      const int col0 = nb * kBN + h * 128;
+      const bool active = col0 < p.N;
       if (!wait_bounded(&sh->acc_full, acc_ph, abort_flag, p.err, kErrSiteGemmAccFull)) break;
       ptx::tc_fence_after();
       uint32_t v[4][32];
@@ -209,12 +220,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_before();
       __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&sh->acc_empty);
+      if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_leader);
       acc_ph ^= 1u;
       if (!active) continue;
       const int row = m0 + q * 32 + lane;
       if (row < p.M) {
-        const int col0 = n0 + h * 128;
         __nv_bfloat16* yrow = p.Y + static_cast<size_t>(row) * p.N + col0;
         const float sc = p.out_scale;
 #pragma unroll
@@ -249,24 +259,69 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
+  // Both CTAs finished: every MMA has completed (each epilogue saw its last
+  // accumulator) and no remote arrive is still in flight.
   ptx::tc_fence_before();
-  __syncthreads();
+  ptx::cluster_sync();
   if (warp == 1) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tmem, kTmemCols);
+    ptx::tmem_dealloc_pair(tmem, kTmemCols);
   }
+}
+
+int max_active_clusters(size_t smem) {
+  static int cache[64] = {0};
+  int dev = 0;
+  cudaGetDevice(&dev);
+  if (dev >= 0 && dev < 64 && cache[dev] > 0) return cache[dev];
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel, &cfg) != cudaSuccess || n <= 0) {
+    cudaGetLastError();
+    return 0;
+  }
+  if (dev >= 0 && dev < 64) cache[dev] = n;
+  return n;
 }
 
 }  // namespace
 
-cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
-                              const CUtensorMap& tl2, const GemmParams& p, int num_sms, cudaStream_t s) {
-  const size_t smem = 1024 + kStages * kStageBytes + sizeof(SharedTail);
+size_t gemm_nvfp4_smem_bytes() { return 1024 + kStages * kStageBytes + sizeof(SharedTail); }
+
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
+                              const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
+                              const GemmParams& p, int num_sms, cudaStream_t s) {
+  const size_t smem = gemm_nvfp4_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  gemm_nvfp4_kernel<<<grid, kThreads, smem, s>>>(ta, tb, tz, tl2, p);
+  int clusters = max_active_clusters(smem);
+  if (clusters <= 0) clusters = num_sms / 2;
+  if (clusters > p.num_tiles) clusters = p.num_tiles;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2 * clusters, 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, ta, tb, tsfa, tsfb, tz, tl2, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

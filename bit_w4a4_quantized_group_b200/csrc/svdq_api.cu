@@ -49,6 +49,27 @@ bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int ele
   return r == CUDA_SUCCESS;
 }
 
+// 3-D tensor [d2][d1][d0] (d0 innermost) with byte strides s1, s2, no swizzle.
+bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0, uint64_t d1, uint64_t d2,
+                  uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[3] = {d0, d1, d2};
+  cuuint64_t strides[2] = {s1, s2};
+  cuuint32_t box[3] = {b0, b1, b2};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// The 128x4 blocked E4M3 scale layout seen as [rows/128][K/64][64 x 8-byte words]:
+// one TMA box = `blocks` row blocks x 4 groups-of-4 = the scales of 128*blocks rows x 256 columns.
+bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows_pad, int64_t K, uint32_t blocks) {
+  return make_tmap_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT64, 64, static_cast<uint64_t>(K / 64),
+                      static_cast<uint64_t>(rows_pad / 128), 512, static_cast<uint64_t>(K / 64) * 512, 64, 4, blocks);
+}
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
@@ -205,20 +226,22 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
   CUtensorMap tz, tl2;
   cudaError_t e;
   if (fmt == SVDQ_FMT_NVFP4_G16) {
-    p.tiles_m = static_cast<int>((M + 127) / 128);
+    p.tiles_m = static_cast<int>((M + 255) / 256);
     p.tiles_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.tiles_m * p.tiles_n;
-    CUtensorMap ta, tb;
+    CUtensorMap ta, tb, tsfa, tsfb;
     if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) return SVDQ_ERR_CUDA;
-    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 256)) return SVDQ_ERR_CUDA;
+    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) return SVDQ_ERR_CUDA;
+    if (!make_tmap_sf(&tsfa, a_scales, p.Mpad, K, 1)) return SVDQ_ERR_CUDA;
+    if (!make_tmap_sf(&tsfb, w_scales, p.Npad, K, 2)) return SVDQ_ERR_CUDA;
     if (rank > 0) {
       if (!make_tmap(&tz, Z_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, M, 64, 128)) return SVDQ_ERR_CUDA;
-      if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 256)) return SVDQ_ERR_CUDA;
+      if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 128)) return SVDQ_ERR_CUDA;
     } else {
       tz = ta;
       tl2 = tb;
     }
-    e = launch_gemm_nvfp4(ta, tb, tz, tl2, p, sms, static_cast<cudaStream_t>(cuda_stream));
+    e = launch_gemm_nvfp4(ta, tb, tsfa, tsfb, tz, tl2, p, sms, static_cast<cudaStream_t>(cuda_stream));
   } else {
     return SVDQ_ERR_UNSUPPORTED;
   }

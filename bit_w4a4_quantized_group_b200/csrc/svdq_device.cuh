@@ -82,8 +82,10 @@ int prologue_stages(int rank);
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
                             cudaStream_t s);
 
-cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
-                              const CUtensorMap& tl2, const GemmParams& p, int num_sms, cudaStream_t s);
+size_t gemm_nvfp4_smem_bytes();
+cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
+                              const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
+                              const GemmParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_gemm_int4(const CUtensorMap& tz, const CUtensorMap& tl2, const GemmParams& p, int num_sms,
                              cudaStream_t s);
 
