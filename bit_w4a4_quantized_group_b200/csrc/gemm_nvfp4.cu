@@ -21,6 +21,7 @@
 //     ring slots hold Z (bf16) and L2s (bf16): kind::f16 MMAs add Z L2s^T into the
 //     *same* accumulator.  L2s was divided by (g_x g_w) at pack time, so the
 //     epilogue's single multiply by g_x g_w scales both terms and Y is written once;
+//   * a scale-copy warp feeds the scales into two TMEM buffers ahead of the MMAs;
 //   * eight epilogue warps per CTA drain TMEM (tcgen05.ld), release it to the
 //     MMA warp at once, then apply g_x g_w and the bias and store bf16 Y.
 #include <cuda.h>
@@ -37,7 +38,8 @@ constexpr int kBM = 256, kBN = 256;           // pair tile
 constexpr int kRows = 128;                    // A rows (and B rows) per CTA
 constexpr int kKTile = 256;                   // E2M1 elements per pipeline step
 constexpr int kStages = 5;
-constexpr int kThreads = 320;                 // producer, MMA, 8 epilogue warps
+constexpr int kThreads = 352;                 // producer, MMA, scale-copy, 8 epilogue warps
+constexpr int kEpiWarp0 = 3;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = kRows * 128;     // 16 KB
 constexpr uint32_t kBBytes = kRows * 128;     // 16 KB
@@ -48,8 +50,11 @@ constexpr uint32_t kSfbOff = kSfaOff + kSfaBytes;
 constexpr uint32_t kStageBytes = kSfbOff + kSfbBytes;   // 38 KB
 constexpr uint32_t kTxMain = 2 * kStageBytes;            // both CTAs
 constexpr uint32_t kTxLowRank = 2 * (kABytes + kBBytes);
+constexpr uint32_t kEpiBoxBytes = 32 * 128;             // 32 rows x 64 bf16 per epilogue warp
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSfa = 256, kTmemSfb = 272;
+// Scale factors live in two TMEM buffers used by alternate pipeline steps, so that the
+// copies of step k+1 do not wait for the MMAs of step k to stop reading them.
+constexpr uint32_t kTmemSf0 = 256, kTmemSfStride = 48;   // per buffer: SFA 16 columns, SFB 32 columns
 
 __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
   // E2M1 x E2M1, UE4M3 scales, K-major A and B, dense
@@ -67,6 +72,8 @@ struct SharedTail {
   uint64_t empty[kStages];
   uint64_t acc_full;
   uint64_t acc_empty;
+  uint64_t sf_ready[2];     // scale buffer b holds the scales of the current step (copies done)
+  uint64_t sf_free[2];      // the MMAs that read scale buffer b have completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -75,10 +82,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_z, const __grid_constant__ CUtensorMap tmap_l2,
-                      GemmParams p) {
+                      const __grid_constant__ CUtensorMap tmap_y, GemmParams p) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  SharedTail* sh = reinterpret_cast<SharedTail*>(smem + kStages * kStageBytes);
+  uint8_t* epi_smem = smem + kStages * kStageBytes;                       // 8 x 4 KB staging for Y
+  SharedTail* sh = reinterpret_cast<SharedTail*>(epi_smem + kEpiWarps * kEpiBoxBytes);
   volatile int* abort_flag = &sh->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -98,6 +106,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(&sh->acc_full, 1);
     ptx::mbar_init(&sh->acc_empty, 2 * kEpiWarps);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&sh->sf_ready[b], 1);
+      ptx::mbar_init(&sh->sf_free[b], 1);
+    }
     sh->abort_flag = 0;
     ptx::fence_mbar_init();
   }
@@ -150,10 +162,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
     __syncwarp();
+  } else if (warp == 2) {
+    // ------------------------------------------------------------ scale copier (leader CTA only)
+    // Moves each step's block scales smem -> TMEM (both CTAs) into alternating buffers, so
+    // that the copies run beside the MMAs of the previous step instead of in series with them.
+    if (rank == 0) {
+      int it = 0, mi = 0;
+      bool ok = true;
+      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
+        for (int k = 0; k < nk; ++k, ++it) {
+          if (k >= nk_main) continue;
+          const int s = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          const int b = mi & 1;
+          if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull) ||
+              !wait_bounded(&sh->sf_free[b], ((mi >> 1) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmSfFree)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          if (lane == 0) {
+            const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
+            const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
+            const uint32_t sfa = tmem + kTmemSf0 + b * kTmemSfStride;
+            const uint32_t sfb = sfa + 16;
+            for (int kb = 0; kb < nkb; ++kb) {
+              ptx::tmem_cp_32x128b_warpx4_pair(sfa + kb * 4, ptx::sdesc_sf(st + kSfaOff + kb * 512));
+              ptx::tmem_cp_32x128b_warpx4_pair(sfb + kb * 8, ptx::sdesc_sf(st + kSfbOff + kb * 512));
+              ptx::tmem_cp_32x128b_warpx4_pair(sfb + kb * 8 + 4, ptx::sdesc_sf(st + kSfbOff + 2048 + kb * 512));
+            }
+            ptx::tc_commit_pair_local(&sh->sf_ready[b]);
+          }
+          __syncwarp();
+          ++mi;
+        }
+      }
+    }
   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer (leader CTA only)
     if (rank == 0) {
-      int it = 0;
+      int it = 0, mi = 0;
       uint32_t acc_ph = 0;
       bool ok = true;
       const uint32_t id4 = idesc_nvf4(kBM, kBN);
@@ -165,22 +213,24 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
           if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull)) { ok = false; break; }
+          const bool main_step = k < nk_main;
+          const int b = mi & 1;
+          if (main_step && !wait_bounded(&sh->sf_ready[b], (mi >> 1) & 1, abort_flag, p.err, kErrSiteGemmSfReady)) {
+            ok = false;
+            break;
+          }
           ptx::tc_fence_after();
           if (lane == 0) {
             const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
-            if (k < nk_main) {
+            if (main_step) {
               const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
-              for (int kb = 0; kb < nkb; ++kb) {
-                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfa + kb * 4, ptx::sdesc_sf(st + kSfaOff + kb * 512));
-                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfb + kb * 8, ptx::sdesc_sf(st + kSfbOff + kb * 512));
-                ptx::tmem_cp_32x128b_warpx4_pair(tmem + kTmemSfb + kb * 8 + 4,
-                                                 ptx::sdesc_sf(st + kSfbOff + 2048 + kb * 512));
-              }
+              const uint32_t sfa = tmem + kTmemSf0 + b * kTmemSfStride;
+              const uint32_t sfb = sfa + 16;
               for (int kb = 0; kb < nkb; ++kb) {
                 ptx::umma_nvf4_pair(tmem, ptx::sdesc_sw128(st + kb * 32), ptx::sdesc_sw128(st + kABytes + kb * 32),
-                                    id4, tmem + kTmemSfa + kb * 4, tmem + kTmemSfb + kb * 8,
-                                    (k | kb) != 0 ? 1u : 0u);
+                                    id4, sfa + kb * 4, sfb + kb * 8, (k | kb) != 0 ? 1u : 0u);
               }
+              ptx::tc_commit_pair_local(&sh->sf_free[b]);
             } else {
               const int c = k - nk_main;
               const int nmma = min(64, p.rank - c * 64) / 16;
@@ -191,6 +241,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             ptx::tc_commit_pair(&sh->empty[s], 0x3);
           }
           __syncwarp();
+          if (main_step) ++mi;
         }
         if (!ok) break;
         if (lane == 0) ptx::tc_commit_pair(&sh->acc_full, 0x3);
@@ -199,9 +250,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 2-9, both CTAs)
+    // ------------------------------------------------------------ epilogue (warps 3-10, both CTAs)
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
-    const int h = (warp - 2) >> 2;          // column half of the 256-wide tile
+    const int h = (warp - kEpiWarp0) >> 2;  // column half of the 256-wide tile
     const uint32_t acc_empty_leader = ptx::mapa_shared(ptx::smem_u32(&sh->acc_empty), 0);
     uint32_t acc_ph = 0;
     for (int t = cluster; t < p.num_tiles; t += nclusters) {
@@ -223,40 +274,50 @@ __global__ void __launch_bounds__(kThreads, 1)
       if (lane == 0) ptx::mbar_arrive_cluster(acc_empty_leader);
       acc_ph ^= 1u;
       if (!active) continue;
-      const int row = m0 + q * 32 + lane;
-      if (row < p.M) {
-        __nv_bfloat16* yrow = p.Y + static_cast<size_t>(row) * p.N + col0;
-        const float sc = p.out_scale;
+      // Y = g_x g_w * acc + bias -> bf16, staged in 128B-swizzled shared memory (32 rows x 64
+      // columns per box) and written with TMA stores; rows past M are clipped by the tensor map.
+      uint8_t* buf = epi_smem + (warp - kEpiWarp0) * kEpiBoxBytes;
+      const float sc = p.out_scale;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
+      for (int box = 0; box < 2; ++box) {
+        if (lane == 0) ptx::bulk_wait_group_read<0>();
+        __syncwarp();
 #pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) {
-            float bv[8];
-            if (p.bias) {
-              const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + c * 32 + c8 * 8));
-              const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                bv[2 * e] = __uint_as_float(bw[e] << 16);
-                bv[2 * e + 1] = __uint_as_float(bw[e] & 0xFFFF0000u);
-              }
-            } else {
-#pragma unroll
-              for (int e = 0; e < 8; ++e) bv[e] = 0.f;
-            }
-            uint32_t o[4];
+        for (int c8 = 0; c8 < 8; ++c8) {
+          const int cl = box * 64 + c8 * 8;                 // column within this warp's 128
+          float bv[8];
+          if (p.bias) {
+            const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + cl));
+            const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
 #pragma unroll
             for (int e = 0; e < 4; ++e) {
-              const float y0 = fmaf(__uint_as_float(v[c][c8 * 8 + 2 * e]), sc, bv[2 * e]);
-              const float y1 = fmaf(__uint_as_float(v[c][c8 * 8 + 2 * e + 1]), sc, bv[2 * e + 1]);
-              __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
-              o[e] = *reinterpret_cast<uint32_t*>(&hv);
+              bv[2 * e] = __uint_as_float(bw[e] << 16);
+              bv[2 * e + 1] = __uint_as_float(bw[e] & 0xFFFF0000u);
             }
-            *reinterpret_cast<uint4*>(yrow + c * 32 + c8 * 8) = make_uint4(o[0], o[1], o[2], o[3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) bv[e] = 0.f;
           }
+          uint32_t o[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const float y0 = fmaf(__uint_as_float(v[cl / 32][cl % 32 + 2 * e]), sc, bv[2 * e]);
+            const float y1 = fmaf(__uint_as_float(v[cl / 32][cl % 32 + 2 * e + 1]), sc, bv[2 * e + 1]);
+            __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
+            o[e] = *reinterpret_cast<uint32_t*>(&hv);
+          }
+          *reinterpret_cast<uint4*>(buf + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+        }
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::tma_store_2d(&tmap_y, buf, col0 + box * 64, m0 + q * 32);
+          ptx::bulk_commit_group();
         }
       }
     }
+    if (lane == 0) ptx::bulk_wait_group<0>();
+    __syncwarp();
   }
 
   // Both CTAs finished: every MMA has completed (each epilogue saw its last
@@ -296,11 +357,11 @@ int max_active_clusters(size_t smem) {
 
 }  // namespace
 
-size_t gemm_nvfp4_smem_bytes() { return 1024 + kStages * kStageBytes + sizeof(SharedTail); }
+size_t gemm_nvfp4_smem_bytes() { return 1024 + kStages * kStageBytes + kEpiWarps * kEpiBoxBytes + sizeof(SharedTail); }
 
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
                               const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
-                              const GemmParams& p, int num_sms, cudaStream_t s) {
+                              const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s) {
   const size_t smem = gemm_nvfp4_smem_bytes();
   cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
@@ -320,7 +381,7 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, ta, tb, tsfa, tsfb, tz, tl2, p);
+  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, ta, tb, tsfa, tsfb, tz, tl2, ty, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

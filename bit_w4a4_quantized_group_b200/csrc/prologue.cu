@@ -7,14 +7,28 @@
 // divide is X D^-1 of §3.1 eq.(3); the quantizers are eq.(1) (INT4 g64,
 // 16-bit scale) and NVFP4 g16 with E4M3 scales (§2.2, §8).
 //
-// Design (B200): HBM-bound.  A dedicated producer warp streams 32-row x
-// 256-column tiles of X (and the matching 256 columns of L1 and lambda) into
-// a shared-memory ring with TMA; eight compute warps each own a 16-row x
-// 64-column box of every tile.  X_hat is formed in registers in the
-// m16n8k16 fragment layout so that the same registers feed the bf16 tensor-
-// core MMA for Z and the quantizer; codes are staged per warp in shared
-// memory and written back as 16-byte row segments.  Z partials of the four
+// Design (B200, HBM-bound): a producer warp streams 32-row tiles of X (and the
+// matching columns of L1) into a shared-memory ring with TMA, and writes
+// lambda and RN(1/lambda) for the tile's columns next to them.  NW compute
+// warps each own a 16-row x 64-column box of every tile.  X_hat is formed in
+// registers in the m16n8k16 fragment layout, so the same registers feed the
+// bf16 tensor-core MMA for Z and the quantizer; codes are staged per warp in
+// shared memory and written back as 16-byte row segments.  Z partials of the
 // warps that share a row strip are summed in a fixed order (deterministic).
+//
+// Divisions are IEEE-exact without the divide instruction sequence:
+//  * X / lambda uses Markstein's correction (P. Markstein, "Computation of
+//    elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
+//    Dev. 34(1), 1990): with y = RN(1/b) and an approximation q of a/b, the
+//    remainder r = a - b q is exact under FMA and RN(q + r y) = RN(a/b) once q
+//    is within one ulp.  Two correction steps from q0 = RN(a y) are used: the
+//    first brings q within one ulp, the second rounds correctly.
+//  * x_hat / (s g) only decides a 4-bit code: x_hat has 8 significant bits and
+//    (s g) at most 11, so the exact quotient is either exactly a rounding
+//    midpoint of the code grid or at least 2^-16 (relative) away from every
+//    midpoint.  One correction step from an approximate reciprocal recovers
+//    exact midpoints exactly and leaves every other quotient within 2^-20 of
+//    its value, so the code equals the code of the correctly rounded quotient.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -27,21 +41,22 @@ namespace svdq {
 
 namespace {
 
-constexpr int kProThreads = 288;      // 8 compute warps + 1 producer warp
-constexpr int kProRows = 32;          // rows per CTA
-constexpr int kProCols = 256;         // columns per pipeline stage (4 boxes of 64)
+constexpr int kProRows = 32;                      // rows per CTA (two 16-row strips)
 constexpr uint32_t kXBoxBytes = kProRows * 128;   // 32 rows x 64 bf16
 
+__host__ __device__ constexpr int compute_warps(int rank) { return rank <= 64 ? 16 : 8; }
+
 struct ProSmemLayout {
-  uint32_t x_off, l1_off, lam_off, stage_bytes;
+  uint32_t x_off, l1_off, lam_off, rlam_off, stage_bytes;
 };
 
-__host__ __device__ inline ProSmemLayout pro_layout(int rank) {
+__host__ __device__ inline ProSmemLayout pro_layout(int rank, int boxes) {
   ProSmemLayout L;
   L.x_off = 0;
-  L.l1_off = 4 * kXBoxBytes;                       // 16 KB
-  L.lam_off = L.l1_off + 4u * 128u * rank;         // 4 boxes of r rows x 128 B
-  uint32_t sz = L.lam_off + kProCols * 4;          // 1 KB of lambda
+  L.l1_off = boxes * kXBoxBytes;
+  L.lam_off = L.l1_off + boxes * 128u * rank;
+  L.rlam_off = L.lam_off + boxes * 64u * 4u;
+  uint32_t sz = L.rlam_off + boxes * 64u * 4u;
   L.stage_bytes = (sz + 1023u) & ~1023u;
   return L;
 }
@@ -53,58 +68,89 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// RN(a / b) given y = RN(1 / b), b > 0 (two Markstein corrections; sign of a kept for a = -0).
+__device__ __forceinline__ float div_rn(float a, float b, float y) {
+  const float q0 = a * y;
+  const float q1 = fmaf(fmaf(-b, q0, a), y, q0);
+  const float q2 = fmaf(fmaf(-b, q1, a), y, q1);
+  return copysignf(q2, a);
+}
+__device__ __forceinline__ float rcp_approx(float x) {
+  float r;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(x));
+  return r;
+}
+// a / b accurate enough to decide a 4-bit code (see the header), exact on midpoints.
+__device__ __forceinline__ float div_code(float a, float b, float y) {
+  const float q0 = a * y;
+  return copysignf(fmaf(fmaf(-b, q0, a), y, q0), a);
+}
+
 template <int FMT, int RANK>
-__global__ void __launch_bounds__(kProThreads, 1)
+__global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_l1,
                     ProParams p) {
+  constexpr int NW = compute_warps(RANK);      // compute warps
+  constexpr int BOXES = NW / 2;                 // 64-column boxes per stage
+  constexpr int BK = 64 * BOXES;                // columns per stage
   constexpr int NT = RANK / 8;                  // n8 tiles of Z
-  const ProSmemLayout L = pro_layout(RANK);
+  const ProSmemLayout L = pro_layout(RANK, BOXES);
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * L.stage_bytes);
   uint64_t* empty = full + S;
-  uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // 8 warps x 512 B code staging
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(cstage + 8 * 512);
+  uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // NW warps x 512 B code staging
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(cstage + NW * 512);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kProRows;
-  const int nkt = (p.K + kProCols - 1) / kProCols;
+  const int nkt = (p.K + BK - 1) / BK;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full[s], 1);
-      ptx::mbar_init(&empty[s], 8);
+      ptx::mbar_init(&full[s], 32);     // every producer lane arrives (its lambda stores)
+      ptx::mbar_init(&empty[s], NW);
     }
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   __syncthreads();
 
-  if (warp == 8) {
-    // ---------------------------------------------------------------- producer
-    if (ptx::elect_one()) {
+  if (warp == NW) {
+    // ---------------------------------------------------------------- producer warp
+    if (lane == 0) {
       ptx::prefetch_tmap(&tmap_x);
       if (RANK > 0) ptx::prefetch_tmap(&tmap_l1);
-      for (int kt = 0; kt < nkt; ++kt) {
-        const int s = kt % S;
-        const uint32_t ph = (kt / S) & 1;
-        if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
-        const int col0 = kt * kProCols;
-        const int cols = min(kProCols, p.K - col0);
-        const int nbox = cols / 64;
-        uint32_t bytes = nbox * (kXBoxBytes + 128u * RANK) + (p.lam ? cols * 4u : 0u);
-        ptx::mbar_arrive_expect_tx(&full[s], bytes);
-        uint8_t* st = smem + s * L.stage_bytes;
+    }
+    for (int kt = 0; kt < nkt; ++kt) {
+      const int s = kt % S;
+      const uint32_t ph = (kt / S) & 1;
+      if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
+      const int col0 = kt * BK;
+      const int nbox = min(BK, p.K - col0) / 64;
+      uint8_t* st = smem + s * L.stage_bytes;
+      float* lam_s = reinterpret_cast<float*>(st + L.lam_off);
+      float* rlam_s = reinterpret_cast<float*>(st + L.rlam_off);
+#pragma unroll
+      for (int i = 0; i < BK / 32; ++i) {
+        const int c = i * 32 + lane;
+        float l = 1.f;
+        if (p.lam && col0 + c < p.K) l = __ldg(p.lam + col0 + c);
+        lam_s[c] = l;
+        rlam_s[c] = __frcp_rn(l);
+      }
+      if (lane == 0) {
+        ptx::mbar_arrive_expect_tx(&full[s], nbox * (kXBoxBytes + 128u * RANK));
         for (int b = 0; b < nbox; ++b) {
           ptx::tma_load_2d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], col0 + b * 64, m0);
           if (RANK > 0) ptx::tma_load_2d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], col0 + b * 64, 0);
         }
-        if (p.lam) ptx::bulk_load(st + L.lam_off, p.lam + col0, cols * 4u, &full[s]);
+      } else {
+        ptx::mbar_arrive(&full[s]);
       }
     }
-    __syncwarp();
   } else {
     // ---------------------------------------------------------------- compute warps
     const int strip = warp & 1;         // rows 16*strip .. 16*strip+15 of the CTA tile
@@ -118,18 +164,21 @@ __global__ void __launch_bounds__(kProThreads, 1)
     uint8_t* cst = cstage + warp * 512;
     const int K2 = p.K / 2;
     const float gs = p.gscale;
+    const float inv_gs = 1.0f / gs;     // exact: gs is a power of two
+    constexpr float kRcp6 = 1.0f / 6.0f, kRcp7 = 1.0f / 7.0f;
     bool ok = true;
 
     for (int kt = 0; kt < nkt && ok; ++kt) {
       const int s = kt % S;
       const uint32_t ph = (kt / S) & 1;
       if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
-      const int col0 = kt * kProCols + phase * 64;
+      const int col0 = kt * BK + phase * 64;
       if (col0 < p.K) {
         const uint8_t* st = smem + s * L.stage_bytes;
         const uint32_t xbox = ptx::smem_u32(st + L.x_off + phase * kXBoxBytes);
         const uint32_t l1box = ptx::smem_u32(st + L.l1_off + phase * 128 * RANK);
         const float* lam_s = reinterpret_cast<const float*>(st + L.lam_off) + phase * 64;
+        const float* rlam_s = reinterpret_cast<const float*>(st + L.rlam_off) + phase * 64;
         float xv[4][8];                 // X_hat values: [k16 tile][row g: 0..3, row g+8: 4..7]
         uint32_t sc_pack_a = 0, sc_pack_b = 0;
 #pragma unroll
@@ -141,20 +190,16 @@ __global__ void __launch_bounds__(kProThreads, 1)
             ptx::ldmatrix_x4(xbox + r * 128 + ((ch ^ (r & 7)) << 4), a[0], a[1], a[2], a[3]);
           }
           const int c0 = j * 16 + tig * 2;
-          // smoothing divide X / lambda (IEEE fp32), one rounding to bf16
-          float l0 = 1.f, l1 = 1.f, l8 = 1.f, l9 = 1.f;
-          if (p.lam) { l0 = lam_s[c0]; l1 = lam_s[c0 + 1]; l8 = lam_s[c0 + 8]; l9 = lam_s[c0 + 9]; }
+          // smoothing divide X / lambda (IEEE-exact), one rounding to bf16
+          const float2 l01 = *reinterpret_cast<const float2*>(lam_s + c0);
+          const float2 l89 = *reinterpret_cast<const float2*>(lam_s + c0 + 8);
+          const float2 r01 = *reinterpret_cast<const float2*>(rlam_s + c0);
+          const float2 r89 = *reinterpret_cast<const float2*>(rlam_s + c0 + 8);
           uint32_t ah[4];
-          {
-            float x0 = bf16lo(a[0]) / l0, x1 = bf16hi(a[0]) / l1;   // row g,   cols c0, c0+1
-            float x2 = bf16lo(a[1]) / l0, x3 = bf16hi(a[1]) / l1;   // row g+8, cols c0, c0+1
-            float x4 = bf16lo(a[2]) / l8, x5 = bf16hi(a[2]) / l9;   // row g,   cols c0+8, c0+9
-            float x6 = bf16lo(a[3]) / l8, x7 = bf16hi(a[3]) / l9;   // row g+8, cols c0+8, c0+9
-            ah[0] = pack_bf16x2(x0, x1);
-            ah[1] = pack_bf16x2(x2, x3);
-            ah[2] = pack_bf16x2(x4, x5);
-            ah[3] = pack_bf16x2(x6, x7);
-          }
+          ah[0] = pack_bf16x2(div_rn(bf16lo(a[0]), l01.x, r01.x), div_rn(bf16hi(a[0]), l01.y, r01.y));
+          ah[1] = pack_bf16x2(div_rn(bf16lo(a[1]), l01.x, r01.x), div_rn(bf16hi(a[1]), l01.y, r01.y));
+          ah[2] = pack_bf16x2(div_rn(bf16lo(a[2]), l89.x, r89.x), div_rn(bf16hi(a[2]), l89.y, r89.y));
+          ah[3] = pack_bf16x2(div_rn(bf16lo(a[3]), l89.x, r89.x), div_rn(bf16hi(a[3]), l89.y, r89.y));
           xv[j][0] = bf16lo(ah[0]); xv[j][1] = bf16hi(ah[0]);
           xv[j][2] = bf16lo(ah[2]); xv[j][3] = bf16hi(ah[2]);
           xv[j][4] = bf16lo(ah[1]); xv[j][5] = bf16hi(ah[1]);
@@ -177,18 +222,20 @@ __global__ void __launch_bounds__(kProThreads, 1)
             ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-            const uint32_t sa = ptx::cvt_e4m3((ma / 6.0f) / gs);
-            const uint32_t sb = ptx::cvt_e4m3((mb / 6.0f) / gs);
+            const uint32_t sa = ptx::cvt_e4m3(div_rn(ma, 6.0f, kRcp6) * inv_gs);
+            const uint32_t sb = ptx::cvt_e4m3(div_rn(mb, 6.0f, kRcp6) * inv_gs);
             const float da = ptx::e4m3_to_f32(sa) * gs;
             const float db = ptx::e4m3_to_f32(sb) * gs;
             uint32_t qa0 = 0, qa1 = 0, qb0 = 0, qb1 = 0;
             if (da > 0.f) {
-              qa0 = ptx::cvt_e2m1x2(xv[j][0] / da, xv[j][1] / da);
-              qa1 = ptx::cvt_e2m1x2(xv[j][2] / da, xv[j][3] / da);
+              const float ya = rcp_approx(da);
+              qa0 = ptx::cvt_e2m1x2(div_code(xv[j][0], da, ya), div_code(xv[j][1], da, ya));
+              qa1 = ptx::cvt_e2m1x2(div_code(xv[j][2], da, ya), div_code(xv[j][3], da, ya));
             }
             if (db > 0.f) {
-              qb0 = ptx::cvt_e2m1x2(xv[j][4] / db, xv[j][5] / db);
-              qb1 = ptx::cvt_e2m1x2(xv[j][6] / db, xv[j][7] / db);
+              const float yb = rcp_approx(db);
+              qb0 = ptx::cvt_e2m1x2(div_code(xv[j][4], db, yb), div_code(xv[j][5], db, yb));
+              qb1 = ptx::cvt_e2m1x2(div_code(xv[j][6], db, yb), div_code(xv[j][7], db, yb));
             }
             cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(qa0);
             cst[g * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(qa1);
@@ -212,17 +259,20 @@ __global__ void __launch_bounds__(kProThreads, 1)
           ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
           mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
           mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-          const __half ha = __float2half_rn(fminf(ma / 7.0f, 65504.0f));
-          const __half hb = __float2half_rn(fminf(mb / 7.0f, 65504.0f));
+          const __half ha = __float2half_rn(fminf(div_rn(ma, 7.0f, kRcp7), 65504.0f));
+          const __half hb = __float2half_rn(fminf(div_rn(mb, 7.0f, kRcp7), 65504.0f));
           const float fa = __half2float(ha), fb = __half2float(hb);
+          const float ya = fa > 0.f ? rcp_approx(fa) : 0.f;
+          const float yb = fb > 0.f ? rcp_approx(fb) : 0.f;
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t q[8];
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
               const float den = (e < 4) ? fa : fb;
+              const float y = (e < 4) ? ya : yb;
               int v = 0;
-              if (den > 0.f) v = max(-7, min(7, __float2int_rn(xv[j][e] / den)));
+              if (den > 0.f) v = max(-7, min(7, __float2int_rn(div_code(xv[j][e], den, y))));
               q[e] = static_cast<uint32_t>(v) & 0xFu;
             }
             cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(q[0] | (q[1] << 4));
@@ -264,7 +314,7 @@ __global__ void __launch_bounds__(kProThreads, 1)
 
     // ---------------------------------------------------------------- Z = X_hat L1^T
     if (NT > 0) {
-      __syncthreads_compute(ok);
+      named_barrier_sync(1, 32 * NW);
       float* zbuf = reinterpret_cast<float*>(smem);       // [phase][strip][16][RANK]
       float* zb = zbuf + ((phase * 2 + strip) * 16) * RANK;
 #pragma unroll
@@ -275,22 +325,23 @@ __global__ void __launch_bounds__(kProThreads, 1)
         zb[(g + 8) * RANK + c] = acc[nt][2];
         zb[(g + 8) * RANK + c + 1] = acc[nt][3];
       }
-      __syncthreads_compute(ok);
-      // warps of phase 0 sum the four partials in phase order and store bf16
+      named_barrier_sync(1, 32 * NW);
+      // the two warps of phase 0 sum the partials in phase order and store bf16
       if (phase == 0) {
-        for (int idx = lane; idx < 16 * RANK / 2; idx += 32) {
-          const int r = (idx * 2) / (RANK > 0 ? RANK : 1), c = (idx * 2) % (RANK > 0 ? RANK : 1);
+        constexpr int R1 = RANK > 0 ? RANK : 1;
+        for (int idx = lane; idx < 16 * R1 / 2; idx += 32) {
+          const int r = (idx * 2) / R1, c = (idx * 2) % R1;
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-          for (int ph = 0; ph < 4; ++ph) {
-            const float* src = zbuf + ((ph * 2 + strip) * 16 + r) * RANK + c;
+          for (int ph = 0; ph < BOXES; ++ph) {
+            const float* src = zbuf + ((ph * 2 + strip) * 16 + r) * R1 + c;
             s0 += src[0];
             s1 += src[1];
           }
           const int row = m0 + strip * 16 + r;
           if (row < p.M) {
             __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
-            *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * RANK + c) = v;
+            *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * R1 + c) = v;
           }
         }
       }
@@ -298,30 +349,33 @@ __global__ void __launch_bounds__(kProThreads, 1)
   }
 }
 
-}  // namespace
-
-size_t prologue_smem_bytes(int rank, int stages) {
-  const ProSmemLayout L = pro_layout(rank);
-  return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + 8 * 512 + 16;
+template <int RANK>
+size_t smem_bytes_for(int stages) {
+  constexpr int NW = compute_warps(RANK);
+  const ProSmemLayout L = pro_layout(RANK, NW / 2);
+  return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + NW * 512 + 16;
 }
 
-int prologue_stages(int rank) {
-  const ProSmemLayout L = pro_layout(rank);
-  int s = static_cast<int>((200u * 1024u) / L.stage_bytes);
+template <int RANK>
+int stages_for() {
+  constexpr int NW = compute_warps(RANK);
+  const ProSmemLayout L = pro_layout(RANK, NW / 2);
+  const size_t budget = 220 * 1024 - 1024 - NW * 512 - 64;
+  int s = static_cast<int>(budget / L.stage_bytes);
   if (s > 4) s = 4;
-  if (s < 2) s = 2;
   return s;
 }
 
 template <int FMT, int RANK>
-static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
-                              cudaStream_t stream) {
-  const size_t smem = prologue_smem_bytes(RANK, p.stages);
+static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, ProParams p, cudaStream_t stream) {
+  p.stages = stages_for<RANK>();
+  if (p.stages < 2) return cudaErrorInvalidConfiguration;
+  const size_t smem = smem_bytes_for<RANK>(p.stages);
   auto kern = prologue_kernel<FMT, RANK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.Mpad / kProRows;
-  kern<<<grid, kProThreads, smem, stream>>>(tx, tl1, p);
+  kern<<<grid, 32 * (compute_warps(RANK) + 1), smem, stream>>>(tx, tl1, p);
   return cudaGetLastError();
 }
 
@@ -341,6 +395,8 @@ static cudaError_t launch_pro_rank(const CUtensorMap& tx, const CUtensorMap& tl1
     default: return cudaErrorInvalidValue;
   }
 }
+
+}  // namespace
 
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
                             cudaStream_t s) {

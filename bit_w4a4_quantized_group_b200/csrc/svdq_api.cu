@@ -172,7 +172,6 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   p.K = static_cast<int>(K);
   p.rank = rank;
   p.Mpad = static_cast<int>((M + 127) / 128 * 128);
-  p.stages = prologue_stages(rank);
   p.lam = lambda;
   p.gscale = act_gscale;
   p.codes = static_cast<uint8_t*>(a_codes);
@@ -241,7 +240,9 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
       tz = ta;
       tl2 = tb;
     }
-    e = launch_gemm_nvfp4(ta, tb, tsfa, tsfb, tz, tl2, p, sms, static_cast<cudaStream_t>(cuda_stream));
+    CUtensorMap ty;
+    if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
+    e = launch_gemm_nvfp4(ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms, static_cast<cudaStream_t>(cuda_stream));
   } else {
     return SVDQ_ERR_UNSUPPORTED;
   }

@@ -22,6 +22,8 @@ enum : int {
   kErrSiteGemmAccFull = 14,
   kErrSiteGemmConvEmpty = 15,
   kErrSiteGemmConvFull = 16,
+  kErrSiteGemmSfFree = 17,
+  kErrSiteGemmSfReady = 18,
 };
 
 // A wait gives up after this many nanoseconds (~1 s); legitimate waits here
@@ -50,8 +52,10 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   }
 }
 
-// Barrier over the 256 compute threads of the prologue (named barrier 1).
-__device__ __forceinline__ void __syncthreads_compute(bool) { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Named barrier `id` over `count` threads (a multiple of 32).
+__device__ __forceinline__ void named_barrier_sync(int id, int count) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
 
 struct ProParams {
   int M, K, rank, Mpad, stages;
@@ -77,15 +81,13 @@ struct GemmParams {
   int num_tiles, tiles_m, tiles_n;
 };
 
-size_t prologue_smem_bytes(int rank, int stages);
-int prologue_stages(int rank);
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
                             cudaStream_t s);
 
 size_t gemm_nvfp4_smem_bytes();
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
                               const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
-                              const GemmParams& p, int num_sms, cudaStream_t s);
+                              const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
 cudaError_t launch_gemm_int4(const CUtensorMap& tz, const CUtensorMap& tl2, const GemmParams& p, int num_sms,
                              cudaStream_t s);
 

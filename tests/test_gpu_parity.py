@@ -175,3 +175,37 @@ def test_layer_end_to_end_small(fmt, rank):
     # and the layer approximates the unquantized X W + b
     exact = layer.X.astype(np.float64) @ layer.W + layer.bias.astype(np.float64)
     assert rel_fro(Yg, exact) < 0.15
+
+
+def _finite_bf16_values(lo=1e-30, hi=1e30):
+    bits = np.arange(65536, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)
+    a = np.abs(v)
+    keep = np.isfinite(v) & (((a >= lo) & (a <= hi)) | (a == 0))
+    return v[keep]
+
+
+@pytest.mark.parametrize("run", range(4))
+def test_smoothing_divide_exhaustive_over_bf16(run):
+    """X_hat = bf16(fp32(x) / lambda) for every finite bf16 x (|x| in [1e-30, 1e30] or 0)
+    and 16 lambdas per run, read back through Z with a 0/1 selector as L1."""
+    rng = np.random.default_rng(1000 + run)
+    special = np.array([1.0, 3.0, 0.1, 7.0, 1 / 3, 0.99999994, 1.0000001, 2.0 ** -7, 1.9999999, 1e-5, 1e5,
+                        6.0, 0.75, 1.5, 123.456, 0.0123], np.float32)
+    lams = special if run == 0 else np.exp(rng.uniform(np.log(1e-5), np.log(1e5), 16)).astype(np.float32)
+    xs = _finite_bf16_values()
+    M, K, r = len(xs), 128, 16
+    X = np.repeat(xs[:, None], K, axis=1).astype(np.float32)
+    lam = np.ones(K, np.float32)
+    cols = np.arange(16) * 8 + 3
+    lam[cols] = lams
+    L1 = np.zeros((r, K), np.float64)
+    L1[np.arange(16), cols] = 1.0
+    got = run_prologue("int4", X, lam, 1.0, L1)
+    want = O.smooth_activations(X[:, cols], lam[cols])
+    Zg = got["Z"]
+    bad = ~((Zg == want) | (np.isnan(Zg) & np.isnan(want)))
+    # -0 and +0 compare equal above; check the sign bit too where it can be observed
+    # (a zero comes back through the fp32 accumulator of Z as +0 whatever its sign)
+    bad |= (np.signbit(Zg) != np.signbit(want)) & (want != 0)
+    assert not bad.any(), f"{bad.sum()} mismatches, first x={X[np.argwhere(bad)[0][0], 0]}"
