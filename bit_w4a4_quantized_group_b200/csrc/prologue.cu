@@ -68,12 +68,13 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
-// RN(a / b) given y = RN(1 / b), b > 0 (two Markstein corrections; sign of a kept for a = -0).
+// RN(a / b) given y = RN(1 / b), b > 0 (two Markstein corrections).
+// The remainder is formed as (b q - a) and subtracted, which keeps the sign of a
+// zero quotient: for a = -0 every step stays -0.
 __device__ __forceinline__ float div_rn(float a, float b, float y) {
   const float q0 = a * y;
-  const float q1 = fmaf(fmaf(-b, q0, a), y, q0);
-  const float q2 = fmaf(fmaf(-b, q1, a), y, q1);
-  return copysignf(q2, a);
+  const float q1 = fmaf(-fmaf(b, q0, -a), y, q0);
+  return fmaf(-fmaf(b, q1, -a), y, q1);
 }
 __device__ __forceinline__ float rcp_approx(float x) {
   float r;
@@ -83,7 +84,7 @@ __device__ __forceinline__ float rcp_approx(float x) {
 // a / b accurate enough to decide a 4-bit code (see the header), exact on midpoints.
 __device__ __forceinline__ float div_code(float a, float b, float y) {
   const float q0 = a * y;
-  return copysignf(fmaf(fmaf(-b, q0, a), y, q0), a);
+  return fmaf(-fmaf(b, q0, -a), y, q0);
 }
 
 template <int FMT, int RANK>
@@ -110,7 +111,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      ptx::mbar_init(&full[s], 32);     // every producer lane arrives (its lambda stores)
+      ptx::mbar_init(&full[s], 32);     // every producer lane arrives (its lambda stores) + TMA bytes
       ptx::mbar_init(&empty[s], NW);
     }
     *abort_flag = 0;
@@ -133,23 +134,26 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       uint8_t* st = smem + s * L.stage_bytes;
       float* lam_s = reinterpret_cast<float*>(st + L.lam_off);
       float* rlam_s = reinterpret_cast<float*>(st + L.rlam_off);
-#pragma unroll
-      for (int i = 0; i < BK / 32; ++i) {
-        const int c = i * 32 + lane;
-        float l = 1.f;
-        if (p.lam && col0 + c < p.K) l = __ldg(p.lam + col0 + c);
-        lam_s[c] = l;
-        rlam_s[c] = __frcp_rn(l);
-      }
+      // TMA first, so that the lambda loads below overlap its latency
       if (lane == 0) {
-        ptx::mbar_arrive_expect_tx(&full[s], nbox * (kXBoxBytes + 128u * RANK));
+        ptx::mbar_expect_tx(&full[s], nbox * (kXBoxBytes + 128u * RANK));
         for (int b = 0; b < nbox; ++b) {
           ptx::tma_load_2d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], col0 + b * 64, m0);
           if (RANK > 0) ptx::tma_load_2d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], col0 + b * 64, 0);
         }
-      } else {
-        ptx::mbar_arrive(&full[s]);
       }
+      float lv[BK / 32];
+#pragma unroll
+      for (int i = 0; i < BK / 32; ++i) {           // independent loads, all in flight together
+        const int c = col0 + i * 32 + lane;
+        lv[i] = (p.lam != nullptr && c < p.K) ? __ldg(p.lam + c) : 1.f;
+      }
+#pragma unroll
+      for (int i = 0; i < BK / 32; ++i) {
+        lam_s[i * 32 + lane] = lv[i];
+        rlam_s[i * 32 + lane] = __frcp_rn(lv[i]);
+      }
+      ptx::mbar_arrive(&full[s]);   // each lane releases its own lambda stores
     }
   } else {
     // ---------------------------------------------------------------- compute warps
