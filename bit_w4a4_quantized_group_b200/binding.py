@@ -22,7 +22,7 @@ FORMATS = {"nvfp4": SVDQ_FMT_NVFP4_G16, "int4": SVDQ_FMT_INT4_G64}
 EXPORTED = (
     "svdq_buffer_sizes", "svdq_pack_weight", "svdq_quantize_act_lowrank_down",
     "svdq_w4a4_gemm_lowrank_up", "svdq_status_string", "svdq_get_last_device_error",
-    "svdq_last_launch_count",
+    "svdq_last_launch_count", "svdq_last_cuda_error",
 )
 
 
@@ -33,7 +33,8 @@ class svdq_sizes(ctypes.Structure):
 
 class SvdqError(RuntimeError):
     def __init__(self, status: int, what: str):
-        super().__init__(f"{what}: {status_name(status)} ({status})")
+        detail = f" [{svdq_last_cuda_error()}]" if status == SVDQ_ERR_CUDA else ""
+        super().__init__(f"{what}: {status_name(status)} ({status}){detail}")
         self.status = status
 
 
@@ -59,8 +60,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_status_string.restype = ctypes.c_char_p
     lib.svdq_get_last_device_error.argtypes = [vp, ctypes.POINTER(c_int)]
     lib.svdq_last_launch_count.argtypes = []
+    lib.svdq_last_cuda_error.argtypes = []
+    lib.svdq_last_cuda_error.restype = ctypes.c_char_p
     for name in EXPORTED:
-        if name not in ("svdq_status_string",):
+        if name not in ("svdq_status_string", "svdq_last_cuda_error"):
             getattr(lib, name).restype = c_int
     _lib = lib
     return lib
@@ -108,6 +111,10 @@ def svdq_get_last_device_error(stream=None):
 
 def svdq_last_launch_count() -> int:
     return load().svdq_last_launch_count()
+
+
+def svdq_last_cuda_error() -> str:
+    return load().svdq_last_cuda_error().decode()
 
 
 # ----------------------------------------------------------------- torch helpers

@@ -19,6 +19,12 @@ __device__ int g_device_error = 0;   // the library's one piece of device state 
 namespace {
 
 thread_local int t_last_launch_count = 0;
+thread_local cudaError_t t_last_cuda_error = cudaSuccess;
+
+svdq_status cuda_fail(cudaError_t e) {
+  t_last_cuda_error = e;
+  return SVDQ_ERR_CUDA;
+}
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
@@ -34,9 +40,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
 }
 
 // 2-D row-major tensor [outer][inner] of `elem` bytes per element, tiled with a
-// box of box_inner x box_outer elements and 128-byte swizzle.
+// box of box_inner x box_outer elements (128-byte swizzle unless stated).
 bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int elem, uint64_t inner,
-               uint64_t outer, uint32_t box_inner, uint32_t box_outer) {
+               uint64_t outer, uint32_t box_inner, uint32_t box_outer,
+               CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_128B) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[2] = {inner, outer};
@@ -44,8 +51,7 @@ bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int ele
   cuuint32_t box[2] = {box_inner, box_outer};
   cuuint32_t estr[2] = {1, 1};
   CUresult r = fn(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -130,6 +136,8 @@ extern "C" svdq_status svdq_buffer_sizes(svdq_format fmt, int64_t M, int64_t N, 
 
 extern "C" int svdq_last_launch_count(void) { return t_last_launch_count; }
 
+extern "C" const char* svdq_last_cuda_error(void) { return cudaGetErrorName(t_last_cuda_error); }
+
 extern "C" svdq_status svdq_get_last_device_error(void* cuda_stream, int* site) {
   if (site) *site = 0;
   if (cudaStreamSynchronize(static_cast<cudaStream_t>(cuda_stream)) != cudaSuccess) return SVDQ_ERR_CUDA;
@@ -181,7 +189,7 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   if (!p.err) return SVDQ_ERR_CUDA;
   cudaError_t e = launch_prologue(fmt == SVDQ_FMT_NVFP4_G16 ? kFmtNvfp4 : kFmtInt4, tx, tl1, p,
                                   static_cast<cudaStream_t>(cuda_stream));
-  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   t_last_launch_count = 1;
   return SVDQ_OK;
 }
@@ -244,9 +252,33 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
     if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
     e = launch_gemm_nvfp4(ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms, static_cast<cudaStream_t>(cuda_stream));
   } else {
-    return SVDQ_ERR_UNSUPPORTED;
+    p.tiles_m = static_cast<int>((M + 127) / 128);
+    p.tiles_n = static_cast<int>(N / 128);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    CUtensorMap ty, ta, tb;
+    if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
+    if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ERR_CUDA;
+    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 64, 128, CU_TENSOR_MAP_SWIZZLE_64B))
+      return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+      if (!make_tmap(&tz, Z_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, M, 64, 128)) return SVDQ_ERR_CUDA;
+      if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 128)) return SVDQ_ERR_CUDA;
+    } else {
+      tz = ta;
+      tl2 = tb;
+    }
+    // group scales: fp16 [K/64][rows_pad] tensors, boxes of 128 rows x 2 groups
+    CUtensorMap tsa, tsb;
+    if (!make_tmap(&tsa, a_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.Mpad, K / 64, 128, 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return SVDQ_ERR_CUDA;
+    if (!make_tmap(&tsb, w_scales, CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 2, p.Npad, K / 64, 128, 2,
+                   CU_TENSOR_MAP_SWIZZLE_NONE))
+      return SVDQ_ERR_CUDA;
+    e = launch_gemm_int4(ta, tb, tz, tl2, ty, tsa, tsb, p, sms, static_cast<cudaStream_t>(cuda_stream));
   }
-  if (e != cudaSuccess) return SVDQ_ERR_CUDA;
+  if (e != cudaSuccess) return cuda_fail(e);
   t_last_launch_count = 1;
   return SVDQ_OK;
 }

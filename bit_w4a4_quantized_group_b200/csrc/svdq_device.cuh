@@ -88,7 +88,9 @@ size_t gemm_nvfp4_smem_bytes();
 cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
                               const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
                               const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
-cudaError_t launch_gemm_int4(const CUtensorMap& tz, const CUtensorMap& tl2, const GemmParams& p, int num_sms,
-                             cudaStream_t s);
+size_t gemm_int4_smem_bytes();
+cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
+                             const CUtensorMap& tl2, const CUtensorMap& ty, const CUtensorMap& tsa,
+                             const CUtensorMap& tsb, const GemmParams& p, int num_sms, cudaStream_t s);
 
 }  // namespace svdq

@@ -168,6 +168,10 @@ svdq_status svdq_get_last_device_error(void* cuda_stream, int* site);
 /* Number of kernels the last successful device call launched (for launch accounting). */
 int svdq_last_launch_count(void);
 
+/* Name of the CUDA runtime error behind the last SVDQ_ERR_CUDA returned on this
+ * host thread ("cudaSuccess" if none). */
+const char* svdq_last_cuda_error(void);
+
 #ifdef __cplusplus
 }
 #endif

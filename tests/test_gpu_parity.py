@@ -123,19 +123,22 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     return Yg, ref
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
 @pytest.mark.parametrize("M,N,K,rank", [(300, 640, 640, 32), (256, 512, 512, 16), (128, 256, 256, 0),
                                         (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64)])
-def test_gemm_parity_nvfp4(M, N, K, rank):
-    _gemm_case("nvfp4", M, N, K, rank, seed=11 + M + N + rank)
+def test_gemm_parity(fmt, M, N, K, rank):
+    _gemm_case(fmt, M, N, K, rank, seed=11 + M + N + rank)
 
 
-def test_gemm_parity_nvfp4_no_bias():
-    _gemm_case("nvfp4", 160, 512, 512, 32, seed=3, with_bias=False)
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_gemm_parity_no_bias(fmt):
+    _gemm_case(fmt, 160, 512, 512, 32, seed=3, with_bias=False)
 
 
-def test_gemm_lowrank_branch_is_added_nvfp4():
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+def test_gemm_lowrank_branch_is_added(fmt):
     """Y(r) - Y(r=0 on the same 4-bit operands) equals Z L2 (the branch really lands in Y)."""
-    fmt, M, N, K, rank = "nvfp4", 128, 256, 256, 32
+    M, N, K, rank = 128, 256, 256, 32
     layer, prep = _layer(M, K, N, rank, seed=19, fmt=fmt)
     gx = prep["act_gscale"]
     packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
@@ -149,7 +152,8 @@ def test_gemm_lowrank_branch_is_added_nvfp4():
     assert rel_fro(Y1 - Y0, branch) < 2e-2
 
 
-@pytest.mark.parametrize("fmt,rank", [("nvfp4", 32), ("nvfp4", 0), ("nvfp4", 128)])
+@pytest.mark.parametrize("fmt,rank", [("nvfp4", 32), ("nvfp4", 0), ("nvfp4", 128), ("int4", 32), ("int4", 0),
+                                      ("int4", 128)])
 def test_layer_end_to_end_small(fmt, rank):
     """Prologue then GEMM on the device (Z never leaves the GPU) vs the reference layer."""
     M, K, N = 384, 768, 768
@@ -209,3 +213,23 @@ def test_smoothing_divide_exhaustive_over_bf16(run):
     # (a zero comes back through the fp32 accumulator of Z as +0 whatever its sign)
     bad |= (np.signbit(Zg) != np.signbit(want)) & (want != 0)
     assert not bad.any(), f"{bad.sum()} mismatches, first x={X[np.argwhere(bad)[0][0], 0]}"
+
+
+def test_tiny_layer_int4_end_to_end():
+    """The tiny INT4 layer (256 x 512 x 512, rank 16, 8 outlier channels x 50) through both calls."""
+    cfg = I.TINY
+    layer = I.make_layer(cfg)
+    fmt = "int4"
+    prep = O.prepare_layer(fmt, layer.X, layer.W, cfg.rank)
+    pk = B.pack_weight_np(fmt, prep["R_nk"], prep["L1_rk"].astype(np.float32), prep["L2_nr"].astype(np.float32), 1.0)
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], 1.0)
+    got = _check_prologue(fmt, layer.X, prep["lam"], 1.0, packed["L1_bf16"])[0]
+    L2s = torch.from_numpy(pk["L2_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    Y = run_gemm(fmt, cfg.b, cfg.n, cfg.m, cfg.rank, got["dev"]["codes"], got["dev"]["scales"], 1.0,
+                 pk["w_codes"], pk["w_scales"], pk["w_gscale"], got["dev"]["Z"], L2s, layer.bias)
+    ref = O.layer_forward(fmt, layer.X, prep["lam"], 1.0, packed, layer.bias)
+    ref_gz = O.gemm_forward(ref["q"], 1.0, packed["q"], 1.0, got["Z"], packed["L2_bf16"], layer.bias)
+    Yg = host_bf16(Y)
+    assert rel_fro(Yg, ref_gz["Y"]) <= Y_TOL
+    exact = layer.X.astype(np.float64) @ layer.W + layer.bias.astype(np.float64)
+    assert rel_fro(Yg, exact) < 0.15
