@@ -50,6 +50,10 @@ def parse_args():
     ap.add_argument("--rank", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--weights", default="svd", choices=["svd", "random"],
+                    help="svd: smoothing + SVD split of the synthetic W (default); random: seeded random "
+                         "R, L1, L2 of the same shapes and scale, no decomposition (for short profiler runs; "
+                         "the kernels' time and traffic do not depend on the weight values)")
     return ap.parse_args()
 
 
@@ -73,64 +77,137 @@ def workload(args):
     return cfg
 
 
-def prepare_layer(cfg, fmt, device):
+def prepare_layer(cfg, fmt, device, weights="svd"):
     from bit_w4a4_quantized_group_b200 import inputs as I
     from bit_w4a4_quantized_group_b200 import prepare as P
     layer = I.make_layer(cfg)
-    prep = P.prepare(fmt, layer.X, layer.W, cfg.rank, device=device)
+    if weights == "svd":
+        prep = P.prepare(fmt, layer.X, layer.W, cfg.rank, device=device)
+    else:
+        rng = np.random.default_rng(cfg.seed + 1000)
+        K, N, r = cfg.m, cfg.n, cfg.rank
+        lam = np.ones(K, np.float32)
+        xa = float(np.abs(layer.X).max())
+        prep = {"lam": lam,
+                "R_nk": (rng.standard_normal((N, K)) * cfg.sigma_w).astype(np.float32),
+                "L1_rk": (rng.standard_normal((r, K)) * 0.05).astype(np.float32),
+                "L2_nr": (rng.standard_normal((N, r)) * 0.05).astype(np.float32),
+                "act_gscale": P.pow2_tensor_scale(xa) if fmt == "nvfp4" else 1.0}
     packed = P.pack(fmt, prep)
     return layer, prep, packed
 
 
 class ClockSampler:
-    """nvidia-smi clocks and throttle reasons sampled every 200 ms while running."""
+    """SM clocks and throttle reasons of one GPU, sampled while the timed steps run.
+
+    Polls NVML from a thread every 5 ms (one sample right at start and one at
+    stop, so even a region of a few milliseconds has samples); falls back to
+    `nvidia-smi -lms 200` if NVML cannot be used.
+    """
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    NAMES = ("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap")
 
-    def __init__(self, gpu_index):
+    def __init__(self, gpu_index, uuid=None, pci=None, period_s=0.005):
         self.gpu = gpu_index
-        self.proc = None
-        self.path = None
+        self.uuid = uuid
+        self.pci = pci
+        self.period = period_s
+        self.samples = []          # (sm_mhz, max_mhz, reasons bitmask names)
+        self.proc = self.path = self.thread = None
+        self._stop = None
+
+    def _nvml_handle(self):
+        """The NVML handle of this process's CUDA device (by UUID, then PCI id; CUDA_VISIBLE_DEVICES
+        renumbers devices, so the CUDA index is the last resort)."""
+        import pynvml as N
+        N.nvmlInit()
+        if self.uuid:
+            try:
+                u = self.uuid if self.uuid.startswith("GPU-") else "GPU-" + self.uuid
+                return N, N.nvmlDeviceGetHandleByUUID(u)
+            except Exception:
+                pass
+        if self.pci:
+            try:
+                return N, N.nvmlDeviceGetHandleByPciBusId(self.pci)
+            except Exception:
+                pass
+        return N, N.nvmlDeviceGetHandleByIndex(self.gpu)
 
     def start(self):
+        import threading
+        try:
+            N, h = self._nvml_handle()
+            bits = {"hw_slowdown": N.nvmlClocksEventReasonHwSlowdown,
+                    "hw_thermal_slowdown": N.nvmlClocksEventReasonHwThermalSlowdown,
+                    "sw_thermal_slowdown": N.nvmlClocksEventReasonSwThermalSlowdown,
+                    "sw_power_cap": N.nvmlClocksEventReasonSwPowerCap}
+            mx = float(N.nvmlDeviceGetMaxClockInfo(h, N.NVML_CLOCK_SM))
+
+            def sample():
+                sm = float(N.nvmlDeviceGetClockInfo(h, N.NVML_CLOCK_SM))
+                r = int(N.nvmlDeviceGetCurrentClocksEventReasons(h))
+                self.samples.append((sm, mx, tuple(n for n, b in bits.items() if r & b)))
+
+            self._stop = threading.Event()
+            sample()
+
+            def loop():
+                while not self._stop.wait(self.period):
+                    sample()
+                sample()
+
+            self.thread = threading.Thread(target=loop, daemon=True)
+            self.thread.start()
+            self.source = "nvml"
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
                  "-lms", "200", "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+            self.source = "nvidia-smi"
         except Exception:
             self.proc = None
 
-    def stop(self):
-        if self.proc is None:
-            return None
+    def _read_smi(self):
         time.sleep(0.25)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
         except Exception:
             self.proc.kill()
-        rows = []
         try:
             with open(self.path) as f:
                 for line in f:
                     parts = [p.strip() for p in line.split(",")]
-                    if len(parts) >= 9:
-                        rows.append(parts)
+                    if len(parts) >= 9 and parts[1].replace(".", "").isdigit():
+                        self.samples.append((float(parts[1]), float(parts[2]),
+                                             tuple(self.NAMES[i] for i in range(4)
+                                                   if parts[5 + i].lower() == "active")))
             os.unlink(self.path)
         except Exception:
+            pass
+
+    def stop(self):
+        if self.thread is not None:
+            self._stop.set()
+            self.thread.join(timeout=5)
+        elif self.proc is not None:
+            self._read_smi()
+        if not self.samples:
             return None
-        if not rows:
-            return None
-        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
-        busy = [s for s in sm if mx and s > 0.5 * max(mx)] or sm
-        return {"sm_mhz": statistics.median(busy) if busy else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        mx = max(s[1] for s in self.samples)
+        sm = [s[0] for s in self.samples]
+        busy = [v for v in sm if v > 0.5 * mx] or sm
+        reasons = sorted({n for s in self.samples for n in s[2]})
+        return {"sm_mhz": statistics.median(busy), "sm_max_mhz": mx, "reasons": reasons,
+                "samples": len(self.samples), "source": self.source}
 
 
 def source_hash(path):
@@ -154,29 +231,44 @@ def recorded_traffic(kernel_src, workload_name):
 
 # ----------------------------------------------------------------------------- CPU reference timing
 
-def time_oracle(cfg, fmt, prep, X, budget_s=15.0, min_rows=16, max_rows=256):
-    """The CPU reference forward (prologue + GEMM, fp64) on a sample of rows."""
-    import oracle as O
+def _oracle_cores():
     try:
         from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
+        return max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
     except Exception:
-        cores = os.cpu_count() or 1
+        return os.cpu_count() or 1
+
+
+def time_oracle(cfg, fmt, prep, X, budget_s=12.0):
+    """The CPU reference forward (prologue + GEMM, fp64 NumPy) on a bounded sample of rows.
+
+    The row count doubles until one call takes about a quarter of the budget (or covers
+    the whole batch); calls of that size then repeat until the budget is spent.
+    """
+    import oracle as O
+    cores = _oracle_cores()
     packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], prep["act_gscale"])
-    rows = min_rows
-    t0 = time.perf_counter()
-    O.layer_forward(fmt, X[:rows], prep["lam"], prep["act_gscale"], packed, None)
-    dt = time.perf_counter() - t0
-    # grow the sample towards ~budget_s of CPU work
-    while dt * 2 < budget_s and rows * 2 <= max_rows:
-        rows *= 2
+    rows = 64
+
+    def run(n, lo=0):
         t0 = time.perf_counter()
-        O.layer_forward(fmt, X[:rows], prep["lam"], prep["act_gscale"], packed, None)
-        dt = time.perf_counter() - t0
-    tflops = 2.0 * rows * cfg.n * cfg.m / dt / 1e12
+        O.layer_forward(fmt, X[lo:lo + n], prep["lam"], prep["act_gscale"], packed, None)
+        return time.perf_counter() - t0
+
+    dt = run(rows)
+    while dt * 4 < budget_s and rows * 2 <= cfg.b:
+        rows *= 2
+        dt = run(rows)
+    total, calls, done = dt, 1, rows
+    while total < budget_s:
+        lo = (calls * rows) % max(1, cfg.b - rows + 1)
+        total += run(rows, lo)
+        calls += 1
+        done += rows
+    tflops = 2.0 * done * cfg.n * cfg.m / total / 1e12
     return {"value": tflops, "unit": UNIT, "cores": cores, "kind": "oracle",
-            "sample": f"{rows} of {cfg.b} rows of {cfg.name} ({fmt}, r={cfg.rank}); prologue + GEMM in fp64 "
-                      f"NumPy, {dt:.2f} s"}, packed
+            "sample": f"{calls} calls x {rows} of {cfg.b} rows of {cfg.name} ({fmt}, r={cfg.rank}); "
+                      f"prologue + GEMM in fp64 NumPy, {total:.1f} s"}, packed
 
 
 def run_reference(args):
@@ -191,22 +283,18 @@ def run_reference(args):
     prep = {"lam": prep["lam"], "R_nk": prep["R_nk"], "L1_rk": prep["L1_rk"], "L2_nr": prep["L2_nr"],
             "act_gscale": prep["act_gscale"]}
     packed = O.pack_weight(args.format, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], prep["act_gscale"])
-    rows = 16
+    rows = min(512, cfg.b)
     for _ in range(args.warmup):
         O.layer_forward(args.format, layer.X[:rows], prep["lam"], prep["act_gscale"], packed, None)
     times = []
     for i in range(args.steps):
-        lo = (i * rows) % cfg.b
+        lo = (i * rows) % (cfg.b - rows + 1)
         t0 = time.perf_counter()
         O.layer_forward(args.format, layer.X[lo:lo + rows], prep["lam"], prep["act_gscale"], packed, None)
         times.append(time.perf_counter() - t0)
     t = sum(times) / len(times)
     value = 2.0 * rows * cfg.n * cfg.m / t / 1e12
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] + [1])
-    except Exception:
-        cores = os.cpu_count() or 1
+    cores = _oracle_cores()
     out = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
@@ -254,7 +342,7 @@ def main():
 
     cfg = workload(args)
     fmt = args.format
-    layer, prep, packed = prepare_layer(cfg, fmt, str(device))
+    layer, prep, packed = prepare_layer(cfg, fmt, str(device), args.weights)
     M, K, N, r = cfg.b, cfg.m, cfg.n, cfg.rank
     lin = W4A4LowRankLinear(fmt, N, K, packed, prep["lam"], prep["act_gscale"], layer.bias, device=device)
     from bit_w4a4_quantized_group_b200.inputs import bf16_bits
@@ -277,11 +365,16 @@ def main():
     if st != B.SVDQ_OK:
         raise RuntimeError(f"device error {st} at site {site}")
 
-    clocks = ClockSampler(local)
-    clocks.start()
+    props = torch.cuda.get_device_properties(local)
+    pci = None
+    if hasattr(props, "pci_bus_id"):
+        pci = f"{props.pci_domain_id:08X}:{props.pci_bus_id:02X}:{props.pci_device_id:02X}.0"
+    clocks = ClockSampler(local, uuid=str(getattr(props, "uuid", "")) or None, pci=pci)
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
     launches = 0
     barrier()
+    clocks.start()
+    torch.cuda.nvtx.range_push("svdq_timed")
     for i in range(args.steps):
         flush.zero_()
         ev[i][0].record(stream)
@@ -292,6 +385,7 @@ def main():
         launches += B.svdq_last_launch_count()
         ev[i][2].record(stream)
     barrier()
+    torch.cuda.nvtx.range_pop()
     clk = clocks.stop()
     t_pro = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps * 1e-3
     t_gemm = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps * 1e-3
@@ -367,7 +461,8 @@ def main():
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": fmt, "data": "synthetic",
+        "vs_baseline": None, "dtype": fmt,
+        "data": "synthetic" if args.weights == "svd" else "synthetic, random weights (no SVD split)",
         "config": config_dict(cfg, fmt, "flushed: 512 MB write between timed steps, outside the events"),
         "roofline": {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                      "frac": achieved / peak, "traffic": traffic, "kernel": f"gemm_{fmt}",
