@@ -11,16 +11,23 @@
 // B200 design (one CTA per SM, 128 x 128 output tiles, persistent):
 //   * a producer warp streams the packed codes of 128-column K steps into a
 //     3-deep ring with TMA (64B-swizzled, so the row reads below are free of
-//     bank conflicts); four widening warps turn every code into an E4M3 byte
-//     (each integer in -7..7 is exact in E4M3) in the 128B-swizzled K-major
-//     layout of the MMA, in a second 3-deep ring;
-//   * the MMA warp issues tcgen05 kind::f8f6f4 MMAs (E4M3 x E4M3 -> fp32) per
-//     64-element group into one of four TMEM group buffers, so D_g comes out of
-//     the tensor cores as an exact fp32 integer;
-//   * eight epilogue warps drain each group buffer, release it at once, and add
-//     D_g * (s_x s_w) in fp32 into register accumulators; the low-rank branch is
-//     one more "group" (bf16 kind::f16 MMAs, scale 1) whose Z and L2 tiles the
-//     producer loads with TMA into their own slot;
+//     bank conflicts); four widening warps turn every code q into the int8 byte
+//     16 q in the 128B-swizzled K-major layout of the MMA, in a second 3-deep
+//     ring.  A nibble moved to the top of its byte *is* 16 q in two's complement,
+//     so eight codes take two logic operations: the even nibbles of a 32-bit word
+//     go to one word, the odd ones to the next.  That permutes K inside every
+//     8-element chunk, identically for A and B, which leaves each group's dot
+//     product unchanged;
+//   * the MMA warp issues tcgen05 kind::i8 MMAs (s8 x s8 -> s32) per 64-element
+//     group into one of four TMEM group buffers.  Each buffer is preset to the
+//     bit pattern of the float 1.5 * 2^23, so after the MMAs it holds the fp32
+//     number 1.5 * 2^23 + 256 D_g exactly (|256 D_g| <= 2^20): subtracting
+//     1.5 * 2^23 recovers 256 D_g exactly without an int-to-float conversion;
+//   * eight epilogue warps drain each group buffer, preset it again, release it,
+//     and add 256 D_g * (s_x s_w / 256) in fp32 into register accumulators with
+//     packed f32x2 operations (the products and sums are those of D_g * s_x s_w);
+//     the low-rank branch is one more "group" (bf16 kind::f16 MMAs, scale 1)
+//     whose Z and L2 tiles the producer loads with TMA into their own slot;
 //   * Y leaves through 128B-swizzled shared-memory boxes and TMA stores.
 // The per-group fp32 scaling is CUDA-core work of the same order as the MMAs;
 // it is what the INT4 format costs next to NVFP4, whose group scales the
@@ -52,11 +59,12 @@ constexpr uint32_t kScBytes = 1024;            // s_x: 2 groups x 128 rows, s_w:
 constexpr uint32_t kEpiBoxBytes = 32 * 128;    // 32 rows x 64 bf16
 constexpr int kGroupBufs = 4;                  // TMEM: 4 x 128 fp32 columns
 
-__host__ __device__ constexpr uint32_t idesc_e4m3(int m, int n) {
-  // E4M3 x E4M3 -> fp32, K-major A and B
-  return (1u << 4) | (0u << 7) | (0u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
+__host__ __device__ constexpr uint32_t idesc_s8(int m, int n) {
+  // s8 x s8 -> s32, K-major A and B
+  return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
 }
+constexpr uint32_t kAccBias = 0x4B400000u;    // bits of 1.5 * 2^23
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
@@ -77,31 +85,10 @@ struct SharedTail {
   int abort_flag;
 };
 
-// Eight 4-bit two's complement codes (low nibble first) -> eight E4M3 bytes.
-// Byte lookup with prmt: one table for codes 0..7, one for 8..15 (= -8..-1),
-// and a per-byte select on the code's sign bit.
-__device__ __forceinline__ uint2 int4x8_to_e4m3x8(uint32_t w) {
-  // E4M3 of 0..7 and of -8..-1
-  constexpr uint32_t kPos0 = 0x44403800u, kPos1 = 0x4E4C4A48u;   // 0,1,2,3 | 4,5,6,7
-  constexpr uint32_t kNeg0 = 0xCACCCED0u, kNeg1 = 0xB8C0C4C8u;   // -8,-7,-6,-5 | -4,-3,-2,-1
-  // nibbles in element order: e0..e7 = bits [4i, 4i+4); put (e0,e2,e4,e6) and (e1,e3,e5,e7) in bytes
-  const uint32_t even = w & 0x0F0F0F0Fu;          // e0, e2, e4, e6 as bytes
-  const uint32_t odd = (w >> 4) & 0x0F0F0F0Fu;    // e1, e3, e5, e7 as bytes
-  // interleave into element order: lo = e0 e1 e2 e3, hi = e4 e5 e6 e7
-  const uint32_t lo = __byte_perm(even, odd, 0x5140);
-  const uint32_t hi = __byte_perm(even, odd, 0x7362);
-  uint2 out;
-  // selectors: byte index (low 3 bits of each code) for the lookup
-  const uint32_t sl = (lo & 0x07u) | ((lo >> 4) & 0x70u) | ((lo >> 8) & 0x700u) | ((lo >> 12) & 0x7000u);
-  const uint32_t sh = (hi & 0x07u) | ((hi >> 4) & 0x70u) | ((hi >> 8) & 0x700u) | ((hi >> 12) & 0x7000u);
-  const uint32_t pl = __byte_perm(kPos0, kPos1, sl), nl = __byte_perm(kNeg0, kNeg1, sl);
-  const uint32_t ph = __byte_perm(kPos0, kPos1, sh), nh = __byte_perm(kNeg0, kNeg1, sh);
-  // sign masks: 0xFF in byte i when code bit 3 is set
-  const uint32_t ml = ((lo >> 3) & 0x01010101u) * 0xFFu;
-  const uint32_t mh = ((hi >> 3) & 0x01010101u) * 0xFFu;
-  out.x = (pl & ~ml) | (nl & ml);
-  out.y = (ph & ~mh) | (nh & mh);
-  return out;
+// Eight 4-bit two's complement codes (low nibble first) -> eight int8 bytes 16 q:
+// .x = codes 0, 2, 4, 6 and .y = codes 1, 3, 5, 7 (the K permutation described above).
+__device__ __forceinline__ uint2 int4x8_to_s8x8_x16(uint32_t w) {
+  return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
 }
 
 __global__ void __launch_bounds__(kThreads, 1)
@@ -158,6 +145,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  if (warp >= kEpiWarp0) {
+    // preset every group buffer (this warp's 32 lanes x 64 columns of each) to the bias pattern
+    const uint32_t base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + ((warp - kEpiWarp0) >> 2) * 64;
+#pragma unroll
+    for (int b = 0; b < kGroupBufs; ++b) {
+      ptx::tmem_st_32x32b_x32_same(base + b * kBN, kAccBias);
+      ptx::tmem_st_32x32b_x32_same(base + b * kBN + 32, kAccBias);
+    }
+    ptx::tmem_wait_st();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -239,8 +239,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint2 ea[4], eb[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            ea[j] = int4x8_to_e4m3x8(wa[j]);
-            eb[j] = int4x8_to_e4m3x8(wb[j]);
+            ea[j] = int4x8_to_s8x8_x16(wa[j]);
+            eb[j] = int4x8_to_s8x8_x16(wb[j]);
           }
           const int c0 = 2 * i, c1 = 2 * i + 1;
           *reinterpret_cast<uint4*>(arow_s + ((c0 ^ (r & 7)) << 4)) = make_uint4(ea[0].x, ea[0].y, ea[1].x, ea[1].y);
@@ -256,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ MMA issuer
     int it = 0, gi = 0, li = 0;
     bool ok = true;
-    const uint32_t id8 = idesc_e4m3(kBM, kBN);
+    const uint32_t id8 = idesc_s8(kBM, kBN);
     const uint32_t id16 = idesc_bf16(kBM, kBN);
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
       for (int k = 0; k < nk_main && ok; ++k, ++it) {
@@ -279,7 +279,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               const uint32_t off = j * 64 + kk * 32;
-              ptx::umma_f8(d, ptx::sdesc_sw128(st + off), ptx::sdesc_sw128(st + kOpBytes + off), id8, kk);
+              // accumulate onto the preset bias pattern (see the header)
+              ptx::umma_i8(d, ptx::sdesc_sw128(st + off), ptx::sdesc_sw128(st + kOpBytes + off), id8, 1u);
             }
             ptx::tc_commit(&sh->grp_full[b]);
           }
@@ -326,9 +327,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
       const int m0 = (t % p.tiles_m) * kBM, n0 = (t / p.tiles_m) * kBN;
       const int col0 = n0 + h * 64;
-      float acc[64];
+      float2 acc[32];
 #pragma unroll
-      for (int c = 0; c < 64; ++c) acc[c] = 0.f;
+      for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
       bool ok = true;
       const int ngroups = G + (p.rank > 0 ? 1 : 0);
       for (int g = 0; g < ngroups; ++g, ++gi) {
@@ -342,12 +343,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             ok = false;
             break;
           }
-          // this warp's 64 column scales of group g, as fp32 in shared memory
+          // this warp's 64 column scales of group g divided by 256 (exact), as fp32 in shared memory
           const uint8_t* sc = sc_smem + ss * kScBytes + (g & 1) * 256;
           const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
           sa = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + lane) * 2));
           __syncwarp();
-          *reinterpret_cast<float2*>(sb_s + 2 * lane) = fb;
+          *reinterpret_cast<float2*>(sb_s + 2 * lane) = make_float2(fb.x * 0.00390625f, fb.y * 0.00390625f);
           __syncwarp();
         }
         const int b = gi % kGroupBufs;
@@ -357,35 +358,36 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t base = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kBN + h * 64;
-        uint32_t v[32];
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
+          uint32_t v[32];
           ptx::tmem_ld_32x32b_x32(base + half * 32, v);
           ptx::tmem_wait_ld();
-          if (half == 1) {
-            // both halves are in registers: hand the buffer back to the MMA warp
-            ptx::tc_fence_before();
-            __syncwarp();
-            if (lane == 0) {
-              ptx::mbar_arrive(&sh->grp_empty[b]);
-              if (!lowrank && (g & 1) == 1) ptx::mbar_arrive(&sh->sc_empty[ss]);
-            }
-          }
           if (lowrank) {
 #pragma unroll
-            for (int c = 0; c < 32; ++c) acc[half * 32 + c] += __uint_as_float(v[c]);
+            for (int c = 0; c < 16; ++c)
+              acc[half * 16 + c] = __fadd2_rn(acc[half * 16 + c],
+                                              make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
           } else {
+            const float2 sa2 = make_float2(sa, sa);
+            const float2 nb2 = make_float2(-12582912.f, -12582912.f);
 #pragma unroll
-            for (int c4 = 0; c4 < 8; ++c4) {
-              const float4 s4 = *reinterpret_cast<const float4*>(sb_s + half * 32 + 4 * c4);
-              const float sv[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-              for (int u = 0; u < 4; ++u) {
-                const int c = 4 * c4 + u;
-                acc[half * 32 + c] = fmaf(__uint_as_float(v[c]), sa * sv[u], acc[half * 32 + c]);
-              }
+            for (int c = 0; c < 16; ++c) {
+              const float2 sb2 = *reinterpret_cast<const float2*>(sb_s + half * 32 + 2 * c);
+              const float2 d = __fadd2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), nb2);
+              acc[half * 16 + c] = __ffma2_rn(d, __fmul2_rn(sa2, sb2), acc[half * 16 + c]);
             }
           }
+          // this half is consumed: preset it again for the buffer's next use
+#pragma unroll
+          for (int c8 = 0; c8 < 4; ++c8) ptx::tmem_st_32x32b_x8_same(base + half * 32 + c8 * 8, kAccBias);
+        }
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          ptx::mbar_arrive(&sh->grp_empty[b]);
+          if (!lowrank && (g & 1) == 1) ptx::mbar_arrive(&sh->sc_empty[ss]);
         }
       }
       sc_it += nk_main;
@@ -411,7 +413,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t o[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
-          __nv_bfloat162 hv = __floats2bfloat162_rn(acc[c8 * 8 + 2 * u] + bv[2 * u], acc[c8 * 8 + 2 * u + 1] + bv[2 * u + 1]);
+          const float2 a2 = acc[c8 * 4 + u];
+          __nv_bfloat162 hv = __floats2bfloat162_rn(a2.x + bv[2 * u], a2.y + bv[2 * u + 1]);
           o[u] = *reinterpret_cast<uint32_t*>(&hv);
         }
         *reinterpret_cast<uint4*>(buf + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);

@@ -131,6 +131,15 @@ def test_gemm_parity(fmt, M, N, K, rank):
 
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("M,N,K,rank", [(2304, 3072, 512, 32), (2560, 2560, 256, 0), (2304, 3072, 256, 128),
+                                        (1300, 3072, 768, 16)])
+def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
+    """More output tiles than resident CTAs (clusters), so each persistent CTA drains several
+    accumulators; short K (one to three pipeline steps per tile) and a two-step branch."""
+    _gemm_case(fmt, M, N, K, rank, seed=5 + M + K + rank)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
 def test_gemm_parity_no_bias(fmt):
     _gemm_case(fmt, 160, 512, 512, 32, seed=3, with_bias=False)
 
