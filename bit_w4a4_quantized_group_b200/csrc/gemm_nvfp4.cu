@@ -9,13 +9,16 @@
 //     with tcgen05 cta_group::2 MMAs (M = 256: each CTA holds 128 rows of A and
 //     128 rows of B; the pair's tensor cores share the B halves, which halves
 //     the shared-memory operand traffic per SM against a one-CTA 128 x 256 tile);
-//   * persistent clusters walk the tile list; K is staged 256 E2M1 elements
-//     (128 bytes per row) at a time through a 5-deep TMA ring per CTA.  Every
-//     load is a TMA tile load into the issuing CTA's own shared memory whose
-//     completion is counted on the leader CTA's barrier (no multicast loads);
+//   * persistent clusters each take a contiguous run of tiles, N fastest; K is
+//     staged 256 E2M1 elements (128 bytes per row) at a time through a 5-deep
+//     TMA ring per CTA.  Every load is a TMA tile load into the issuing CTA's
+//     own shared memory whose completion is counted on the leader CTA's barrier
+//     (no multicast loads);
 //   * block scales (E4M3, one per 16 elements) are TMA-loaded as 512-byte
-//     "128 rows x 4 groups" blocks and moved to TMEM with tcgen05.cp; each CTA
-//     holds its 128 rows of A-scales and all 256 columns of B-scales;
+//     "128 rows x 4 groups" blocks and moved to TMEM with tcgen05.cp by a copy
+//     warp into four rotating scale buffers, so the copies of a step can run up
+//     to three steps ahead of the MMAs that read them; each CTA holds its 128
+//     rows of A-scales and all 256 columns of B-scales;
 //   * the leader's MMA warp issues kind::mxf4nvf4 block-scaled MMAs into an fp32
 //     TMEM accumulator and then ceil(r/64) extra pipeline steps in which the
 //     ring slots hold Z (bf16) and L2s (bf16): kind::f16 MMAs add Z L2s^T into the
@@ -52,9 +55,10 @@ constexpr uint32_t kTxMain = 2 * kStageBytes;            // both CTAs
 constexpr uint32_t kTxLowRank = 2 * (kABytes + kBBytes);
 constexpr uint32_t kEpiBoxBytes = 32 * 128;             // 32 rows x 64 bf16 per epilogue warp
 constexpr uint32_t kTmemCols = 512;
-// Scale factors live in two TMEM buffers used by alternate pipeline steps, so that the
-// copies of step k+1 do not wait for the MMAs of step k to stop reading them.
-constexpr uint32_t kTmemSf0 = 256, kTmemSfStride = 48;   // per buffer: SFA 16 columns, SFB 32 columns
+// TMEM columns: accumulator [0, 256); four scale buffers of 48 columns from 256 (A-scales 16,
+// B-scales 32), used round-robin by the main steps.
+constexpr int kSfBufs = 4;
+constexpr uint32_t kTmemSf0 = 256, kTmemSfStride = 48;
 
 __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
   // E2M1 x E2M1, UE4M3 scales, K-major A and B, dense
@@ -67,13 +71,26 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
+// Tile schedule: cluster c takes the contiguous run [begin, begin + count) of the N-fastest
+// tile numbering, so consecutive tiles of a cluster share the M block.
+struct TileSeq {
+  int begin, count, tiles_n;
+  __device__ TileSeq(int num_tiles, int tiles_n_, int cluster, int nclusters) : tiles_n(tiles_n_) {
+    const int base = num_tiles / nclusters, extra = num_tiles % nclusters;
+    begin = cluster * base + min(cluster, extra);
+    count = base + (cluster < extra ? 1 : 0);
+  }
+  __device__ int mb(int j) const { return (begin + j) / tiles_n; }
+  __device__ int nb(int j) const { return (begin + j) % tiles_n; }
+};
+
 struct SharedTail {
   uint64_t full[kStages];
   uint64_t empty[kStages];
   uint64_t acc_full;
   uint64_t acc_empty;
-  uint64_t sf_ready[2];     // scale buffer b holds the scales of the current step (copies done)
-  uint64_t sf_free[2];      // the MMAs that read scale buffer b have completed
+  uint64_t sf_ready[kSfBufs];  // scale buffer b holds the scales of its step (copies done)
+  uint64_t sf_free[kSfBufs];   // the MMAs that read scale buffer b have completed
   uint32_t tmem_base;
   int abort_flag;
 };
@@ -98,6 +115,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int nk_lr = (p.rank + 63) / 64;
   const int nk = nk_main + nk_lr;
   const int kblk64 = p.K / 64;
+  const TileSeq tiles(p.num_tiles, p.tiles_n, cluster, nclusters);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -106,7 +124,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ptx::mbar_init(&sh->acc_full, 1);
     ptx::mbar_init(&sh->acc_empty, 2 * kEpiWarps);
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < kSfBufs; ++b) {
       ptx::mbar_init(&sh->sf_ready[b], 1);
       ptx::mbar_init(&sh->sf_free[b], 1);
     }
@@ -135,8 +153,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int it = 0;
       bool ok = true;
-      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
-        const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+      for (int j = 0; j < tiles.count && ok; ++j) {
+        const int mb = tiles.mb(j), nb = tiles.nb(j);
         const int m0 = mb * kBM + static_cast<int>(rank) * kRows;     // this CTA's A rows
         const int n0 = nb * kBN;
         const int nb0 = n0 + static_cast<int>(rank) * kRows;          // this CTA's B rows
@@ -169,14 +187,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (rank == 0) {
       int it = 0, mi = 0;
       bool ok = true;
-      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
+      for (int j = 0; j < tiles.count && ok; ++j) {
         for (int k = 0; k < nk; ++k, ++it) {
           if (k >= nk_main) continue;
           const int s = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          const int b = mi & 1;
+          const int b = mi % kSfBufs;
           if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull) ||
-              !wait_bounded(&sh->sf_free[b], ((mi >> 1) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmSfFree)) {
+              !wait_bounded(&sh->sf_free[b], ((mi / kSfBufs) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmSfFree)) {
             ok = false;
             break;
           }
@@ -206,7 +224,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       const uint32_t id4 = idesc_nvf4(kBM, kBN);
       const uint32_t id16 = idesc_bf16(kBM, kBN);
-      for (int t = cluster; t < p.num_tiles && ok; t += nclusters) {
+      for (int j = 0; j < tiles.count && ok; ++j) {
         if (!wait_bounded(&sh->acc_empty, acc_ph ^ 1u, abort_flag, p.err, kErrSiteGemmAccEmpty)) break;
         ptx::tc_fence_after();
         for (int k = 0; k < nk; ++k, ++it) {
@@ -214,8 +232,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t ph = (it / kStages) & 1;
           if (!wait_bounded(&sh->full[s], ph, abort_flag, p.err, kErrSiteGemmFull)) { ok = false; break; }
           const bool main_step = k < nk_main;
-          const int b = mi & 1;
-          if (main_step && !wait_bounded(&sh->sf_ready[b], (mi >> 1) & 1, abort_flag, p.err, kErrSiteGemmSfReady)) {
+          const int b = mi % kSfBufs;
+          if (main_step && !wait_bounded(&sh->sf_ready[b], (mi / kSfBufs) & 1, abort_flag, p.err, kErrSiteGemmSfReady)) {
             ok = false;
             break;
           }
@@ -255,8 +273,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int h = (warp - kEpiWarp0) >> 2;  // column half of the 256-wide tile
     const uint32_t acc_empty_leader = ptx::mapa_shared(ptx::smem_u32(&sh->acc_empty), 0);
     uint32_t acc_ph = 0;
-    for (int t = cluster; t < p.num_tiles; t += nclusters) {
-      const int mb = t % p.tiles_m, nb = t / p.tiles_m;
+    for (int j = 0; j < tiles.count; ++j) {
+      const int mb = tiles.mb(j), nb = tiles.nb(j);
       const int m0 = mb * kBM + static_cast<int>(rank) * kRows;
       const int col0 = nb * kBN + h * 128;
       const bool active = col0 < p.N;
