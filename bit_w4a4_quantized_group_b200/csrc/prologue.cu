@@ -68,6 +68,26 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<uint32_t*>(&h);
 }
 
+// Packed form of the divides below, two lanes at once: the inputs are the negated
+// dividends na = -a and the negated reciprocals ny = -y.  RN(na ny) = RN(a y),
+// fma(b, q, na) = RN(b q - a) and fma(r, ny, q) = RN(q - r y), so every step equals
+// the scalar step bit for bit, signed zeros included, with no negations in the chain.
+__device__ __forceinline__ float2 div_rn2(float2 na, float2 b, float2 ny) {
+  float2 q = __fmul2_rn(na, ny);
+  float2 r = __ffma2_rn(b, q, na);
+  q = __ffma2_rn(r, ny, q);
+  r = __ffma2_rn(b, q, na);
+  return __ffma2_rn(r, ny, q);
+}
+__device__ __forceinline__ float2 div_code2(float2 na, float2 b, float2 ny) {
+  const float2 q = __fmul2_rn(na, ny);
+  return __ffma2_rn(__ffma2_rn(b, q, na), ny, q);
+}
+// -lo and -hi of a bf16 pair as floats
+__device__ __forceinline__ float2 neg_bf16x2(uint32_t v) {
+  return make_float2(__uint_as_float((v << 16) ^ 0x80000000u), __uint_as_float((v & 0xFFFF0000u) ^ 0x80000000u));
+}
+
 // RN(a / b) given y = RN(1 / b), b > 0 (two Markstein corrections).
 // The remainder is formed as (b q - a) and subtracted, which keeps the sign of a
 // zero quotient: for a = -0 every step stays -0.
@@ -108,6 +128,9 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   const int lane = threadIdx.x & 31;
   const int m0 = blockIdx.x * kProRows;
   const int nkt = (p.K + BK - 1) / BK;
+  // Every CTA reads all of L1; starting the K loop at a different stage per CTA spreads
+  // those reads over the L2 instead of sending every SM to the same lines at once.
+  const int kt0 = blockIdx.x % nkt;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -125,10 +148,11 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       ptx::prefetch_tmap(&tmap_x);
       if (RANK > 0) ptx::prefetch_tmap(&tmap_l1);
     }
-    for (int kt = 0; kt < nkt; ++kt) {
-      const int s = kt % S;
-      const uint32_t ph = (kt / S) & 1;
+    for (int ki = 0; ki < nkt; ++ki) {
+      const int s = ki % S;
+      const uint32_t ph = (ki / S) & 1;
       if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
+      const int kt = (kt0 + ki) % nkt;
       const int col0 = kt * BK;
       const int nbox = min(BK, p.K - col0) / 64;
       uint8_t* st = smem + s * L.stage_bytes;
@@ -151,7 +175,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) {
         lam_s[i * 32 + lane] = lv[i];
-        rlam_s[i * 32 + lane] = __frcp_rn(lv[i]);
+        rlam_s[i * 32 + lane] = -__frcp_rn(lv[i]);   // negated, for the packed divides
       }
       ptx::mbar_arrive(&full[s]);   // each lane releases its own lambda stores
     }
@@ -172,10 +196,11 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     constexpr float kRcp6 = 1.0f / 6.0f, kRcp7 = 1.0f / 7.0f;
     bool ok = true;
 
-    for (int kt = 0; kt < nkt && ok; ++kt) {
-      const int s = kt % S;
-      const uint32_t ph = (kt / S) & 1;
+    for (int ki = 0; ki < nkt && ok; ++ki) {
+      const int s = ki % S;
+      const uint32_t ph = (ki / S) & 1;
       if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
+      const int kt = (kt0 + ki) % nkt;
       const int col0 = kt * BK + phase * 64;
       if (col0 < p.K) {
         const uint8_t* st = smem + s * L.stage_bytes;
@@ -183,7 +208,8 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
         const uint32_t l1box = ptx::smem_u32(st + L.l1_off + phase * 128 * RANK);
         const float* lam_s = reinterpret_cast<const float*>(st + L.lam_off) + phase * 64;
         const float* rlam_s = reinterpret_cast<const float*>(st + L.rlam_off) + phase * 64;
-        float xv[4][8];                 // X_hat values: [k16 tile][row g: 0..3, row g+8: 4..7]
+        // -X_hat as float pairs: [k16 tile][row g: pairs 0, 1; row g+8: pairs 2, 3]
+        float2 nx[4][4];
         uint32_t sc_pack_a = 0, sc_pack_b = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -197,17 +223,18 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           // smoothing divide X / lambda (IEEE-exact), one rounding to bf16
           const float2 l01 = *reinterpret_cast<const float2*>(lam_s + c0);
           const float2 l89 = *reinterpret_cast<const float2*>(lam_s + c0 + 8);
-          const float2 r01 = *reinterpret_cast<const float2*>(rlam_s + c0);
-          const float2 r89 = *reinterpret_cast<const float2*>(rlam_s + c0 + 8);
+          const float2 n01 = *reinterpret_cast<const float2*>(rlam_s + c0);
+          const float2 n89 = *reinterpret_cast<const float2*>(rlam_s + c0 + 8);
           uint32_t ah[4];
-          ah[0] = pack_bf16x2(div_rn(bf16lo(a[0]), l01.x, r01.x), div_rn(bf16hi(a[0]), l01.y, r01.y));
-          ah[1] = pack_bf16x2(div_rn(bf16lo(a[1]), l01.x, r01.x), div_rn(bf16hi(a[1]), l01.y, r01.y));
-          ah[2] = pack_bf16x2(div_rn(bf16lo(a[2]), l89.x, r89.x), div_rn(bf16hi(a[2]), l89.y, r89.y));
-          ah[3] = pack_bf16x2(div_rn(bf16lo(a[3]), l89.x, r89.x), div_rn(bf16hi(a[3]), l89.y, r89.y));
-          xv[j][0] = bf16lo(ah[0]); xv[j][1] = bf16hi(ah[0]);
-          xv[j][2] = bf16lo(ah[2]); xv[j][3] = bf16hi(ah[2]);
-          xv[j][4] = bf16lo(ah[1]); xv[j][5] = bf16hi(ah[1]);
-          xv[j][6] = bf16lo(ah[3]); xv[j][7] = bf16hi(ah[3]);
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const float2 qq = div_rn2(neg_bf16x2(a[i]), i < 2 ? l01 : l89, i < 2 ? n01 : n89);
+            ah[i] = pack_bf16x2(qq.x, qq.y);
+          }
+          nx[j][0] = neg_bf16x2(ah[0]);
+          nx[j][1] = neg_bf16x2(ah[2]);
+          nx[j][2] = neg_bf16x2(ah[1]);
+          nx[j][3] = neg_bf16x2(ah[3]);
           // low-rank down projection on the tensor cores
 #pragma unroll
           for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
@@ -220,64 +247,77 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           }
           if (FMT == kFmtNvfp4) {
             // one 16-element group per row per k16 tile
-            float ma = fmaxf(fmaxf(fabsf(xv[j][0]), fabsf(xv[j][1])), fmaxf(fabsf(xv[j][2]), fabsf(xv[j][3])));
-            float mb = fmaxf(fmaxf(fabsf(xv[j][4]), fabsf(xv[j][5])), fmaxf(fabsf(xv[j][6]), fabsf(xv[j][7])));
+            float ma = fmaxf(fmaxf(fabsf(nx[j][0].x), fabsf(nx[j][0].y)), fmaxf(fabsf(nx[j][1].x), fabsf(nx[j][1].y)));
+            float mb = fmaxf(fmaxf(fabsf(nx[j][2].x), fabsf(nx[j][2].y)), fmaxf(fabsf(nx[j][3].x), fabsf(nx[j][3].y)));
             ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
-            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
             mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-            const uint32_t sa = ptx::cvt_e4m3(div_rn(ma, 6.0f, kRcp6) * inv_gs);
-            const uint32_t sb = ptx::cvt_e4m3(div_rn(mb, 6.0f, kRcp6) * inv_gs);
-            const float da = ptx::e4m3_to_f32(sa) * gs;
-            const float db = ptx::e4m3_to_f32(sb) * gs;
+            // s = e4m3(RN(a / 6) / g) for both rows at once (the divide by g is exact)
+            const float2 s6 = div_rn2(make_float2(-ma, -mb), make_float2(6.0f, 6.0f), make_float2(-kRcp6, -kRcp6));
+            const uint32_t sab = ptx::cvt_e4m3x2(s6.x * inv_gs, s6.y * inv_gs);
+            const float2 dab = ptx::e4m3x2_to_f32x2(sab);
+            const float da = dab.x * gs, db = dab.y * gs;
             uint32_t qa0 = 0, qa1 = 0, qb0 = 0, qb1 = 0;
             if (da > 0.f) {
-              const float ya = rcp_approx(da);
-              qa0 = ptx::cvt_e2m1x2(div_code(xv[j][0], da, ya), div_code(xv[j][1], da, ya));
-              qa1 = ptx::cvt_e2m1x2(div_code(xv[j][2], da, ya), div_code(xv[j][3], da, ya));
+              const float2 dd = make_float2(da, da);
+              const float ny = -rcp_approx(da);
+              const float2 nyy = make_float2(ny, ny);
+              const float2 q0 = div_code2(nx[j][0], dd, nyy), q1 = div_code2(nx[j][1], dd, nyy);
+              qa0 = ptx::cvt_e2m1x2(q0.x, q0.y);
+              qa1 = ptx::cvt_e2m1x2(q1.x, q1.y);
             }
             if (db > 0.f) {
-              const float yb = rcp_approx(db);
-              qb0 = ptx::cvt_e2m1x2(div_code(xv[j][4], db, yb), div_code(xv[j][5], db, yb));
-              qb1 = ptx::cvt_e2m1x2(div_code(xv[j][6], db, yb), div_code(xv[j][7], db, yb));
+              const float2 dd = make_float2(db, db);
+              const float ny = -rcp_approx(db);
+              const float2 nyy = make_float2(ny, ny);
+              const float2 q2 = div_code2(nx[j][2], dd, nyy), q3 = div_code2(nx[j][3], dd, nyy);
+              qb0 = ptx::cvt_e2m1x2(q2.x, q2.y);
+              qb1 = ptx::cvt_e2m1x2(q3.x, q3.y);
             }
             cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(qa0);
             cst[g * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(qa1);
             cst[(g + 8) * 32 + j * 8 + tig] = static_cast<uint8_t>(qb0);
             cst[(g + 8) * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(qb1);
-            sc_pack_a |= sa << (8 * j);
-            sc_pack_b |= sb << (8 * j);
+            sc_pack_a |= (sab & 0xFFu) << (8 * j);
+            sc_pack_b |= (sab >> 8) << (8 * j);
           }
         }
         if (FMT == kFmtInt4) {
           // one 64-element group per row per box
           float ma = 0.f, mb = 0.f;
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              ma = fmaxf(ma, fabsf(xv[j][e]));
-              mb = fmaxf(mb, fabsf(xv[j][4 + e]));
-            }
+          for (int j = 0; j < 4; ++j) {
+            ma = fmaxf(ma, fmaxf(fmaxf(fabsf(nx[j][0].x), fabsf(nx[j][0].y)), fmaxf(fabsf(nx[j][1].x), fabsf(nx[j][1].y))));
+            mb = fmaxf(mb, fmaxf(fmaxf(fabsf(nx[j][2].x), fabsf(nx[j][2].y)), fmaxf(fabsf(nx[j][3].x), fabsf(nx[j][3].y))));
+          }
           ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
-          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
           mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+          ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
           mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
-          const __half ha = __float2half_rn(fminf(div_rn(ma, 7.0f, kRcp7), 65504.0f));
-          const __half hb = __float2half_rn(fminf(div_rn(mb, 7.0f, kRcp7), 65504.0f));
+          // s = fp16(RN(a / 7)) for both rows at once
+          const float2 s7 = div_rn2(make_float2(-ma, -mb), make_float2(7.0f, 7.0f), make_float2(-kRcp7, -kRcp7));
+          const __half ha = __float2half_rn(fminf(s7.x, 65504.0f));
+          const __half hb = __float2half_rn(fminf(s7.y, 65504.0f));
           const float fa = __half2float(ha), fb = __half2float(hb);
-          const float ya = fa > 0.f ? rcp_approx(fa) : 0.f;
-          const float yb = fb > 0.f ? rcp_approx(fb) : 0.f;
+          const float2 nya = make_float2(fa > 0.f ? -rcp_approx(fa) : 0.f, fa > 0.f ? -rcp_approx(fa) : 0.f);
+          const float2 nyb = make_float2(fb > 0.f ? -rcp_approx(fb) : 0.f, fb > 0.f ? -rcp_approx(fb) : 0.f);
+          const float2 faa = make_float2(fa, fa), fbb = make_float2(fb, fb);
+          // q = clamp(rint(x / s), -7, 7): clamp first (rint is monotonic and +-7 are integers),
+          // then round by adding 1.5 * 2^23, whose low mantissa bits are then q in two's complement
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             uint32_t q[8];
 #pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float den = (e < 4) ? fa : fb;
-              const float y = (e < 4) ? ya : yb;
-              int v = 0;
-              if (den > 0.f) v = max(-7, min(7, __float2int_rn(div_code(xv[j][e], den, y))));
-              q[e] = static_cast<uint32_t>(v) & 0xFu;
+            for (int pi = 0; pi < 4; ++pi) {
+              const bool rb = pi >= 2;
+              float2 qq = make_float2(0.f, 0.f);
+              if (rb ? fb > 0.f : fa > 0.f) qq = div_code2(nx[j][pi], rb ? fbb : faa, rb ? nyb : nya);
+              qq.x = fminf(fmaxf(qq.x, -7.0f), 7.0f);
+              qq.y = fminf(fmaxf(qq.y, -7.0f), 7.0f);
+              qq = __fadd2_rn(qq, make_float2(12582912.0f, 12582912.0f));
+              q[2 * pi] = __float_as_uint(qq.x) & 0xFu;
+              q[2 * pi + 1] = __float_as_uint(qq.y) & 0xFu;
             }
             cst[g * 32 + j * 8 + tig] = static_cast<uint8_t>(q[0] | (q[1] << 4));
             cst[g * 32 + j * 8 + 4 + tig] = static_cast<uint8_t>(q[2] | (q[3] << 4));

@@ -174,6 +174,15 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// 32 lanes x 16 consecutive 32-bit columns -> 16 registers per thread.
+__device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15}, [%16];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+      : "r"(taddr));
+}
 // Store 32 registers to 32 lanes x 32 consecutive columns (all the same value v).
 __device__ __forceinline__ void tmem_st_32x32b_x32_same(uint32_t taddr, uint32_t v) {
   asm volatile(
@@ -241,7 +250,7 @@ __device__ __forceinline__ void ldmatrix_x4(uint32_t saddr, uint32_t& r0, uint32
                : "r"(saddr));
 }
 __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a)[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
@@ -252,7 +261,7 @@ __device__ __forceinline__ void mma_bf16_16816(float (&d)[4], const uint32_t (&a
 // Two fp32 -> packed E2M1 pair, round to nearest even, saturate: lo -> bits 0-3, hi -> bits 4-7.
 __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
   uint32_t out;
-  asm volatile(
+  asm(
       "{\n\t.reg .b8 t;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\t"
       "cvt.u32.u8 %0, t;\n\t}\n"
@@ -263,13 +272,25 @@ __device__ __forceinline__ uint32_t cvt_e2m1x2(float lo, float hi) {
 // fp32 -> E4M3 (round to nearest even, saturate to 448), returned in the low byte.
 __device__ __forceinline__ uint32_t cvt_e4m3(float x) {
   uint16_t out;
-  asm volatile("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(x));
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(0.0f), "f"(x));
   return static_cast<uint32_t>(out & 0xFFu);
+}
+// Two floats -> two E4M3 bytes (satfinite, round to nearest even): lo in bits 0-7, hi in 8-15.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(out) : "f"(hi), "f"(lo));
+  return static_cast<uint32_t>(out);
+}
+// Two E4M3 bytes (bits 0-7, 8-15) -> two floats (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t c) {
+  uint32_t h2;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c & 0xFFFFu)));
+  return __half22float2(*reinterpret_cast<const __half2*>(&h2));
 }
 // E4M3 byte -> fp32 (exact)
 __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   uint32_t h2;
-  asm volatile("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c & 0xFFu)));
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h2) : "h"(static_cast<uint16_t>(c & 0xFFu)));
   return __half2float(__ushort_as_half(static_cast<unsigned short>(h2 & 0xFFFFu)));
 }
 
