@@ -113,6 +113,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
                     ProParams p) {
   constexpr int NW = compute_warps(RANK);      // compute warps
   constexpr int BOXES = NW / 2;                 // 64-column boxes per stage
+  static_assert(BOXES % kProBoxes == 0, "a stage holds whole TMA loads");
   constexpr int BK = 64 * BOXES;                // columns per stage
   constexpr int NT = RANK / 8;                  // n8 tiles of Z
   const ProSmemLayout L = pro_layout(RANK, BOXES);
@@ -148,6 +149,17 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       ptx::prefetch_tmap(&tmap_x);
       if (RANK > 0) ptx::prefetch_tmap(&tmap_l1);
     }
+    // lambda of the next stage is loaded into registers one stage ahead, so that its latency
+    // overlaps the current stage instead of holding back the stage's release
+    float lv[BK / 32];
+    auto load_lambda = [&](int kt) {
+#pragma unroll
+      for (int i = 0; i < BK / 32; ++i) {           // independent loads, all in flight together
+        const int c = kt * BK + i * 32 + lane;
+        lv[i] = (p.lam != nullptr && c < p.K) ? __ldg(p.lam + c) : 1.f;
+      }
+    };
+    load_lambda(kt0 % nkt);
     for (int ki = 0; ki < nkt; ++ki) {
       const int s = ki % S;
       const uint32_t ph = (ki / S) & 1;
@@ -158,24 +170,23 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       uint8_t* st = smem + s * L.stage_bytes;
       float* lam_s = reinterpret_cast<float*>(st + L.lam_off);
       float* rlam_s = reinterpret_cast<float*>(st + L.rlam_off);
-      // TMA first, so that the lambda loads below overlap its latency
       if (lane == 0) {
-        ptx::mbar_expect_tx(&full[s], nbox * (kXBoxBytes + 128u * RANK));
-        for (int b = 0; b < nbox; ++b) {
-          ptx::tma_load_2d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], col0 + b * 64, m0);
-          if (RANK > 0) ptx::tma_load_2d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], col0 + b * 64, 0);
+        // kProBoxes boxes per load; boxes past K are zero-filled and counted like the others
+        const int nload = (nbox + kProBoxes - 1) / kProBoxes;
+        ptx::mbar_expect_tx(&full[s], nload * kProBoxes * (kXBoxBytes + 128u * RANK));
+        for (int b = 0; b < nload * kProBoxes; b += kProBoxes) {
+          ptx::tma_load_3d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], 0, m0, col0 / 64 + b);
+          if (RANK > 0) ptx::tma_load_3d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], 0, 0, col0 / 64 + b);
         }
       }
-      float lv[BK / 32];
+      float cur[BK / 32];
 #pragma unroll
-      for (int i = 0; i < BK / 32; ++i) {           // independent loads, all in flight together
-        const int c = col0 + i * 32 + lane;
-        lv[i] = (p.lam != nullptr && c < p.K) ? __ldg(p.lam + c) : 1.f;
-      }
+      for (int i = 0; i < BK / 32; ++i) cur[i] = lv[i];
+      if (ki + 1 < nkt) load_lambda((kt0 + ki + 1) % nkt);
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) {
-        lam_s[i * 32 + lane] = lv[i];
-        rlam_s[i * 32 + lane] = -__frcp_rn(lv[i]);   // negated, for the packed divides
+        lam_s[i * 32 + lane] = cur[i];
+        rlam_s[i * 32 + lane] = -__frcp_rn(cur[i]);   // negated, for the packed divides
       }
       ptx::mbar_arrive(&full[s]);   // each lane releases its own lambda stores
     }

@@ -57,7 +57,8 @@ bool make_tmap(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int ele
 
 // 3-D tensor [d2][d1][d0] (d0 innermost) with byte strides s1, s2, no swizzle.
 bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint64_t d0, uint64_t d1, uint64_t d2,
-                  uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2) {
+                  uint64_t s1, uint64_t s2, uint32_t b0, uint32_t b1, uint32_t b2,
+                  CUtensorMapSwizzle swz = CU_TENSOR_MAP_SWIZZLE_NONE) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {d0, d1, d2};
@@ -65,7 +66,7 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint
   cuuint32_t box[3] = {b0, b1, b2};
   cuuint32_t estr[3] = {1, 1, 1};
   CUresult r = fn(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                  CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+                  swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS;
 }
 
@@ -168,10 +169,17 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   if (!is_pow2_positive(act_gscale)) return SVDQ_ERR_INVALID_ARG;
   if (fmt == SVDQ_FMT_INT4_G64 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
 
+  // X and L1 seen as [K/64 column blocks][rows][64 columns]: one load brings kProBoxes
+  // 64-column boxes (128B-swizzled) of 32 X rows or of all L1 rows
   CUtensorMap tx, tl1;
-  if (!make_tmap(&tx, X_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, M, 64, 32)) return SVDQ_ERR_CUDA;
+  const uint64_t rs = static_cast<uint64_t>(K) * 2;
+  if (!make_tmap_3d(&tx, X_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, M, K / 64, rs, 128, 64, 32, kProBoxes,
+                    CU_TENSOR_MAP_SWIZZLE_128B))
+    return SVDQ_ERR_CUDA;
   if (rank > 0) {
-    if (!make_tmap(&tl1, L1_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, K, rank, 64, rank)) return SVDQ_ERR_CUDA;
+    if (!make_tmap_3d(&tl1, L1_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 64, rank, K / 64, rs, 128, 64, rank,
+                      kProBoxes, CU_TENSOR_MAP_SWIZZLE_128B))
+      return SVDQ_ERR_CUDA;
   } else {
     tl1 = tx;
   }

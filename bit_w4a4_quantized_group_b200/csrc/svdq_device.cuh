@@ -57,6 +57,8 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
 }
 
+constexpr int kProBoxes = 4;   // 64-column boxes per prologue TMA load
+
 struct ProParams {
   int M, K, rank, Mpad, stages;
   const float* lam;          // nullable
