@@ -308,6 +308,21 @@ def run_reference(args):
     return 0
 
 
+def max_over_ranks(values, device=None):
+    """Element-wise max of per-rank timings: one all_reduce when several ranks run."""
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(v) for v in values], dtype=torch.float64, device=device)
+    if dist.is_available() and dist.is_initialized() and dist.get_world_size() > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return t.tolist()
+
+
+def whole_job_tflops(world, flops_per_rank, seconds):
+    """Throughput of the whole job: every rank processes flops_per_rank in `seconds` (the slowest rank's time)."""
+    return world * flops_per_rank / seconds / 1e12
+
+
 def config_dict(cfg, fmt, l2):
     return {"workload": f"{cfg.name} {cfg.b}x{cfg.m}x{cfg.n} r={cfg.rank} {fmt}", "M": cfg.b, "K": cfg.m,
             "N": cfg.n, "rank": cfg.rank, "format": fmt, "bias": cfg.with_bias, "l2": l2}
@@ -435,14 +450,11 @@ def main():
         e2e = {"t": t_e2e, "h2d": M * K * 2, "d2h": M * N * 2}
 
     # max over ranks
-    vals = torch.tensor([t_step, t_pro, t_gemm, t_gemm0, e2e["t"] if e2e else 0.0], dtype=torch.float64,
-                        device=device)
-    if world > 1:
-        dist.all_reduce(vals, op=dist.ReduceOp.MAX)
-    t_step, t_pro, t_gemm, t_gemm0, t_e2e = vals.tolist()
+    t_step, t_pro, t_gemm, t_gemm0, t_e2e = max_over_ranks(
+        [t_step, t_pro, t_gemm, t_gemm0, e2e["t"] if e2e else 0.0], device=device)
 
     flops = 2.0 * M * N * K
-    value = world * flops / t_step / 1e12
+    value = whole_job_tflops(world, flops, t_step)
     bf16_burst, bf16_sus, hbm, peak_src = peaks()
     if fmt == "nvfp4":
         peak = bf16_burst * 4.0              # dense FP4 = 4 x dense bf16 (nominal ratio 9 : 2.25)
@@ -476,7 +488,7 @@ def main():
         "clocks": clk,
     }
     if e2e:
-        out["e2e"] = {"value": world * flops / t_e2e / 1e12, "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
+        out["e2e"] = {"value": whole_job_tflops(world, flops, t_e2e), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                       "d2h_bytes_per_step": e2e["d2h"]}
     if world == 1 and rank == 0 and not args.no_cpu_baseline:
         cb, _ = time_oracle(cfg, fmt, prep, layer.X)

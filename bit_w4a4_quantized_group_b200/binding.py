@@ -22,7 +22,7 @@ FORMATS = {"nvfp4": SVDQ_FMT_NVFP4_G16, "int4": SVDQ_FMT_INT4_G64}
 EXPORTED = (
     "svdq_buffer_sizes", "svdq_pack_weight", "svdq_quantize_act_lowrank_down",
     "svdq_w4a4_gemm_lowrank_up", "svdq_status_string", "svdq_get_last_device_error",
-    "svdq_last_launch_count", "svdq_last_cuda_error",
+    "svdq_last_launch_count", "svdq_last_cuda_error", "svdq_selftest_bounded_wait",
 )
 
 
@@ -62,6 +62,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.svdq_last_launch_count.argtypes = []
     lib.svdq_last_cuda_error.argtypes = []
     lib.svdq_last_cuda_error.restype = ctypes.c_char_p
+    lib.svdq_selftest_bounded_wait.argtypes = [i64, vp]
     for name in EXPORTED:
         if name not in ("svdq_status_string", "svdq_last_cuda_error"):
             getattr(lib, name).restype = c_int
@@ -107,6 +108,10 @@ def svdq_get_last_device_error(stream=None):
     site = ctypes.c_int(0)
     st = load().svdq_get_last_device_error(stream, ctypes.byref(site))
     return st, site.value
+
+
+def svdq_selftest_bounded_wait(limit_ns: int, stream=None) -> int:
+    return load().svdq_selftest_bounded_wait(int(limit_ns), stream)
 
 
 def svdq_last_launch_count() -> int:

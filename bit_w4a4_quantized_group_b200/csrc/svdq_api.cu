@@ -155,6 +155,18 @@ extern "C" svdq_status svdq_get_last_device_error(void* cuda_stream, int* site) 
   return SVDQ_OK;
 }
 
+extern "C" svdq_status svdq_selftest_bounded_wait(int64_t limit_ns, void* cuda_stream) {
+  t_last_launch_count = 0;
+  if (limit_ns < 1000 || limit_ns > 5000000000ll) return SVDQ_ERR_INVALID_ARG;
+  int* err = device_error_word();
+  if (!err) return SVDQ_ERR_CUDA;
+  cudaError_t e = launch_selftest_bounded_wait(err, static_cast<uint64_t>(limit_ns),
+                                               static_cast<cudaStream_t>(cuda_stream));
+  if (e != cudaSuccess) return cuda_fail(e);
+  t_last_launch_count = 1;
+  return SVDQ_OK;
+}
+
 extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M, int64_t K, int rank,
                                                       const void* X_bf16, const float* lambda, float act_gscale,
                                                       const void* L1_bf16, void* a_codes, void* a_scales,

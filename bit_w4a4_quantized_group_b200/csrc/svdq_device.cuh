@@ -24,6 +24,7 @@ enum : int {
   kErrSiteGemmConvFull = 16,
   kErrSiteGemmSfFree = 17,
   kErrSiteGemmSfReady = 18,
+  kErrSiteSelftest = 90,
 };
 
 // A wait gives up after this many nanoseconds (~1 s); legitimate waits here
@@ -34,7 +35,7 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;
 // records its site in the device error word, raises the CTA's abort flag and
 // returns false; waiters that see the abort flag return false as well.
 __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                             int* err, int site) {
+                                             int* err, int site, uint64_t limit_ns = kWaitLimitNs) {
   const uint32_t a = ptx::smem_u32(bar);
   if (ptx::mbar_try_wait(a, parity)) return true;
   const uint64_t t0 = ptx::globaltimer();
@@ -43,7 +44,7 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
     if (ptx::mbar_try_wait(a, parity)) return true;
     if ((++spins & 63u) == 0) {
       if (*abort_flag) return false;
-      if (ptx::globaltimer() - t0 > kWaitLimitNs) {
+      if (ptx::globaltimer() - t0 > limit_ns) {
         atomicCAS(err, 0, site);
         *abort_flag = 1;
         return false;
@@ -58,6 +59,9 @@ __device__ __forceinline__ void named_barrier_sync(int id, int count) {
 }
 
 constexpr int kProBoxes = 4;   // 64-column boxes per prologue TMA load
+
+// Self-test of the bounded wait: a wait on a barrier nothing arrives at.
+cudaError_t launch_selftest_bounded_wait(int* err, uint64_t limit_ns, cudaStream_t s);
 
 struct ProParams {
   int M, K, rank, Mpad, stages;

@@ -165,6 +165,17 @@ const char* svdq_status_string(svdq_status s);
  */
 svdq_status svdq_get_last_device_error(void* cuda_stream, int* site);
 
+/*
+ * Failure-path self-test: launches one warp that waits on a barrier nothing arrives
+ * at, with the same bounded wait the kernels use but a limit of limit_ns
+ * nanoseconds (1e3 <= limit_ns <= 5e9).  The wait runs out, the kernel records
+ * site 90 in the device error word and returns, leaving the context usable; a
+ * following svdq_get_last_device_error returns SVDQ_ERR_TIMEOUT with *site == 90.
+ * Returns SVDQ_ERR_INVALID_ARG for a limit out of range, SVDQ_ERR_CUDA if the
+ * launch fails.
+ */
+svdq_status svdq_selftest_bounded_wait(int64_t limit_ns, void* cuda_stream);
+
 /* Number of kernels the last successful device call launched (for launch accounting). */
 int svdq_last_launch_count(void);
 

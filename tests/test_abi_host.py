@@ -178,3 +178,9 @@ def test_pack_weight_rejects(lib):
         B.pack_weight_np("nvfp4", R, None, None, 3.0)     # not a power of two
     with pytest.raises(B.SvdqError):
         B.pack_weight_np("int4", R, None, None, 0.5)      # INT4 needs g_x = 1
+
+
+def test_selftest_rejects_limits_out_of_range():
+    # argument checks run before any CUDA call
+    assert B.svdq_selftest_bounded_wait(10, None) == B.SVDQ_ERR_INVALID_ARG
+    assert B.svdq_selftest_bounded_wait(10_000_000_000, None) == B.SVDQ_ERR_INVALID_ARG
