@@ -86,3 +86,26 @@ def rel_fro(a, b) -> float:
     a = np.asarray(a, np.float64)
     b = np.asarray(b, np.float64)
     return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300))
+
+
+def y_elementwise_slack(qa, gx, qw, gw, Z, L2_nr, bias):
+    """Sum of absolute terms of every output element, in fp64: the scale of the fp32
+    accumulation error the GPU may add (g_x g_w |Q(X_hat)| |Q(R)|^T + |Z| |L2|^T + |bias|)."""
+    import oracle as O
+    fmt_g = qa["q"].shape[1] // qa["scale"].shape[1]
+    xa = np.abs(qa["q"] * np.repeat(qa["scale"].astype(np.float64), fmt_g, axis=1))
+    wb = np.abs(qw["q"] * np.repeat(qw["scale"].astype(np.float64), fmt_g, axis=1))
+    S = gx * gw * (xa @ wb.T)
+    if Z is not None and np.asarray(Z).shape[1] > 0:
+        S = S + np.abs(np.asarray(Z, np.float64)) @ np.abs(np.asarray(L2_nr, np.float64)).T
+    if bias is not None:
+        S = S + np.abs(np.asarray(bias, np.float64))[None, :]
+    return S
+
+
+def assert_y_elementwise(Yg, Y64, S):
+    """Every element within one bf16 ulp of the fp64 value plus 2^-16 of its absolute terms."""
+    from layouts import bf16_ulp
+    err = np.abs(np.asarray(Yg, np.float64) - Y64)
+    tol = bf16_ulp(Y64) + 2.0 ** -16 * S
+    assert np.all(err <= tol), f"max excess {np.max(err - tol)} at {np.unravel_index(np.argmax(err - tol), err.shape)}"

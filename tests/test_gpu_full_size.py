@@ -23,7 +23,7 @@ from bit_w4a4_quantized_group_b200 import build as BUILD
 from bit_w4a4_quantized_group_b200 import inputs as I
 from bit_w4a4_quantized_group_b200.layer import W4A4LowRankLinear
 
-from gpu_helpers import check_device_error, dev_bf16, host_bf16, rel_fro
+from gpu_helpers import assert_y_elementwise, check_device_error, dev_bf16, host_bf16, rel_fro, y_elementwise_slack
 from layouts import bf16_ulp, scales_canonical, unpack_codes
 
 pytestmark = pytest.mark.gpu
@@ -85,6 +85,8 @@ def _run_and_check(cfg, fmt, rows=None, seed=4242):
                          layer.bias)
     assert rel_fro(Yg, ref["Y"]) <= 1e-3
     assert rel_fro(Yg, ref["Y64"]) <= 4e-3
+    assert_y_elementwise(Yg, ref["Y64"], y_elementwise_slack(pro["q"], gx, packed["q"], packed["gscale"], Zg,
+                                                             packed["L2_bf16"] if r else None, layer.bias))
 
 
 def _sample_rows(M, seed):

@@ -16,7 +16,8 @@ from bit_w4a4_quantized_group_b200 import binding as B
 from bit_w4a4_quantized_group_b200 import build as BUILD
 from bit_w4a4_quantized_group_b200 import inputs as I
 
-from gpu_helpers import encode_scales, host_bf16, pack_codes_bytes, rel_fro, run_gemm, run_prologue
+from gpu_helpers import (assert_y_elementwise, encode_scales, host_bf16, pack_codes_bytes, rel_fro, run_gemm,
+                         run_prologue, y_elementwise_slack)
 from layouts import bf16_ulp
 
 pytestmark = pytest.mark.gpu
@@ -120,6 +121,8 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     e_64 = rel_fro(Yg, ref["Y64"])
     assert e_ref <= Y_TOL, (e_ref, e_64)
     assert e_64 <= 4e-3
+    assert_y_elementwise(Yg, ref["Y64"], y_elementwise_slack(pro["q"], gx, packed["q"], packed["gscale"], pro["Z"],
+                                                             packed["L2_bf16"], bias))
     return Yg, ref
 
 
