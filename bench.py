@@ -418,6 +418,43 @@ def main():
         gemm0.append((a, b))
     torch.cuda.synchronize()
     t_gemm0 = sum(a.elapsed_time(b) for a, b in gemm0) / len(gemm0) * 1e-3
+    # Fusion: the layer without the branch (prologue and GEMM at rank 0), and the same layer
+    # with an unfused branch as separate passes (msModelSlim's "residual_out +
+    # F.linear(F.linear(x, l1), l2)" form): X / lambda -> bf16, Z = X_hat L1^T, Y += Z L2^T,
+    # the low-rank products on cuBLAS in bf16.  Reported beside the headline, not part of it.
+    fusion = None
+    if r > 0:
+        lam_d = lin.lam if lin.lam is not None else torch.ones(K, device=device)
+        L1d, L2sd = lin.L1, lin.L2
+        up_scale = lin.act_gscale * lin.w_gscale          # L2 is stored divided by g_x g_w
+
+        def branch():
+            xh = (X.float() / lam_d).to(torch.bfloat16)
+            z = xh @ L1d.t()
+            Y.addmm_(z, L2sd.t(), alpha=up_scale)
+
+        res = {"r0": [], "unfused": []}
+        for i in range(args.warmup + max(5, args.steps // 2)):
+            for key in ("r0", "unfused"):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                lin.prologue_only(X, rank=0)
+                lin.gemm_only(M, Y, rank=0)
+                if key == "unfused":
+                    branch()
+                b.record(stream)
+                if i >= args.warmup:
+                    res[key].append((a, b))
+        torch.cuda.synchronize()
+        t_r0 = sum(a.elapsed_time(b) for a, b in res["r0"]) / len(res["r0"]) * 1e-3
+        t_unf = sum(a.elapsed_time(b) for a, b in res["unfused"]) / len(res["unfused"]) * 1e-3
+        # the unfused layer computes the same Y (up to bf16 rounding of its extra passes)
+        Yu = Y.float().clone()
+        lin.forward(X, Y)
+        rel = float((Yu - Y.float()).norm() / Y.float().norm())
+        fusion = {"t_r0": t_r0, "t_unfused": t_unf, "rel": rel}
     lin.forward(X, Y)                        # restore Y with the branch
     st, site = B.svdq_get_last_device_error(None)
     if st != B.SVDQ_OK:
@@ -450,8 +487,9 @@ def main():
         e2e = {"t": t_e2e, "h2d": M * K * 2, "d2h": M * N * 2}
 
     # max over ranks
-    t_step, t_pro, t_gemm, t_gemm0, t_e2e = max_over_ranks(
-        [t_step, t_pro, t_gemm, t_gemm0, e2e["t"] if e2e else 0.0], device=device)
+    t_step, t_pro, t_gemm, t_gemm0, t_e2e, t_r0, t_unf = max_over_ranks(
+        [t_step, t_pro, t_gemm, t_gemm0, e2e["t"] if e2e else 0.0,
+         fusion["t_r0"] if fusion else 0.0, fusion["t_unfused"] if fusion else 0.0], device=device)
 
     flops = 2.0 * M * N * K
     value = whole_job_tflops(world, flops, t_step)
@@ -484,6 +522,12 @@ def main():
         "gemm_frac_fp4_peak": (flops / t_gemm / 1e12) / peak,
         "prologue": {"bound": "hbm", "GB/s": pro_bytes / t_pro / 1e9, "peak": hbm,
                      "frac": pro_bytes / t_pro / 1e9 / hbm, "bytes": pro_bytes},
+        "fusion": None if not fusion else {
+            "layer_r0_us": t_r0 * 1e6, "fused_layer_us": t_step * 1e6,
+            "fused_overhead_pct": 100.0 * (t_step / t_r0 - 1.0),
+            "unfused_layer_us": t_unf * 1e6, "unfused_overhead_pct": 100.0 * (t_unf / t_r0 - 1.0),
+            "unfused_branch": "torch bf16 passes: X/lambda, Z = X_hat L1^T, Y += Z L2^T (cuBLAS)",
+            "unfused_vs_fused_rel_fro": fusion["rel"]},
         "gpu_launches": launches,
         "clocks": clk,
     }

@@ -70,8 +70,10 @@ class W4A4LowRankLinear:
                                  self.act_gscale, self.w_codes, self.w_scales, self.w_gscale,
                                  ws["Z"] if r else None, self.L2 if r else None, self.bias, Y)
 
-    def prologue_only(self, X: torch.Tensor):
+    def prologue_only(self, X: torch.Tensor, rank: Optional[int] = None):
+        """The prologue alone (rank 0 quantizes without the down projection)."""
         M, _ = X.shape
         ws = self.workspace(M)
-        B.quantize_act_lowrank_down_t(self.fmt, X, self.lam, self.act_gscale, self.L1,
-                                      ws["a_codes"], ws["a_scales"], ws["Z"])
+        r = self.rank if rank is None else rank
+        B.quantize_act_lowrank_down_t(self.fmt, X, self.lam, self.act_gscale, self.L1 if r else None,
+                                      ws["a_codes"], ws["a_scales"], ws["Z"] if r else None)

@@ -45,6 +45,11 @@ Readings where the pages are silent (each one is listed in the design doc):
    to bf16); it feeds both the quantizer and the down projection.  L1, L2 and
    Z are bf16.
 8. Sigma goes into L1 (eq.(10) of *SVDQuant 阅读笔记*).
+9. MXFP4 (*AutoRound SVDQuant*, the Nunchaku export: "MXFP4 E2M1 W4A4, group size 32,
+   symmetric"): the MX shared scale of the OCP Microscaling format,
+   ``X = 2 ** clip(floor(log2(amax)) - 2, -127, 127)`` (2 = exponent of the largest
+   E2M1 value 6), stored as its E8M0 byte ``log2(X) + 127``; ``q = e2m1_rn_satfinite(x / X)``
+   (the divide is exact).  ``amax == 0`` gives byte 0.  No tensor scale (g = 1).
 """
 from __future__ import annotations
 
@@ -60,12 +65,13 @@ __all__ = [
     "lora_concat", "pow2_global_scale", "quantize_int4_g64", "quantize_nvfp4_g16",
     "dequantize", "quantize", "prologue", "pack_weight", "w4a4_main", "gemm_forward",
     "layer_forward", "prepare_layer", "rho_mac", "rho_bytes", "prop41_bound",
-    "brute_force_w4a4", "INT4_QMAX", "NVFP4_QMAX", "E4M3_MAX",
+    "brute_force_w4a4", "INT4_QMAX", "NVFP4_QMAX", "E4M3_MAX", "quantize_mxfp4_g32", "MXFP4_EMAX",
 ]
 
 INT4_QMAX = 7          # eq.(1): symmetric codes -7..7
 NVFP4_QMAX = 6.0       # largest E2M1 magnitude
 E4M3_MAX = 448.0       # largest finite E4M3 magnitude
+MXFP4_EMAX = 2         # exponent of the largest E2M1 magnitude: 6 = 1.5 * 2^2
 
 
 # ---------------------------------------------------------------------------
@@ -306,16 +312,37 @@ def quantize_nvfp4_g16(x: np.ndarray, gscale: float):
             "scale": s.astype(np.float32), "scale_bits": s_bits, "gscale": float(gscale)}
 
 
+def quantize_mxfp4_g32(x: np.ndarray):
+    """MXFP4 per 32-element group with a shared power-of-two (E8M0) scale (reading 9).
+
+    X = 2^clip(floor(log2 a) - 2, -127, 127), a = max |x| of the group; q = e2m1(x / X).
+    """
+    x = np.asarray(x, dtype=np.float32)
+    rows, K = x.shape
+    xg = x.reshape(rows, K // 32, 32)
+    a = np.max(np.abs(xg), axis=2).astype(np.float64)
+    mant, ex = np.frexp(a)                     # a = mant * 2^ex, mant in [0.5, 1): floor(log2 a) = ex - 1
+    e = np.where(a > 0, ex - 1 - MXFP4_EMAX, -127)
+    e = np.clip(e, -127, 127).astype(np.int64)
+    X = np.ldexp(1.0, e)                       # exact powers of two
+    v = (xg.astype(np.float64) / X[..., None]).astype(np.float32)   # exact: division by 2^e
+    codes, vals = e2m1_rn_satfinite(v)
+    return {"codes": codes.reshape(rows, K).astype(np.uint8), "q": vals.reshape(rows, K).astype(np.float64),
+            "scale": X, "scale_bits": (e + 127).astype(np.uint8), "gscale": 1.0}
+
+
 def quantize(fmt: str, x: np.ndarray, gscale: float = 1.0):
     if fmt == "int4":
         return quantize_int4_g64(x)
     if fmt == "nvfp4":
         return quantize_nvfp4_g16(x, gscale)
+    if fmt == "mxfp4":
+        return quantize_mxfp4_g32(x)
     raise ValueError(fmt)
 
 
 def group_size(fmt: str) -> int:
-    return 64 if fmt == "int4" else 16
+    return {"int4": 64, "nvfp4": 16, "mxfp4": 32}[fmt]
 
 
 def dequantize(fmt: str, qd) -> np.ndarray:
@@ -361,7 +388,7 @@ def pack_weight(fmt: str, R_nk: np.ndarray, L1_rk: np.ndarray, L2_nr: np.ndarray
     if fmt == "nvfp4":
         gw = pow2_global_scale(np.max(np.abs(R_nk)) if R_nk.size else 0.0)
     else:
-        gw = 1.0
+        gw = 1.0      # INT4 and MXFP4 have no tensor scale
     qd = quantize(fmt, R_nk, gw)
     L1b = bf16_rn(L1_rk)
     L2b = bf16_rn(L2_nr)

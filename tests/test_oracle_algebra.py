@@ -119,7 +119,7 @@ def test_cancellation_eq8(tiny):
 
 
 def test_prop41_bound_eq6(tiny):
-    for fmt in ("int4", "nvfp4"):
+    for fmt in ("int4", "nvfp4", "mxfp4"):
         lam = O.smoothing_factors(tiny.X, tiny.W)
         xh = O.smooth_activations(tiny.X, lam)
         Wt = O.smooth_weight(tiny.W, lam).astype(np.float32)
@@ -131,7 +131,7 @@ def test_prop41_bound_eq6(tiny):
         assert lhs <= mid * (1 + 1e-12) and mid <= rhs * (1 + 1e-12)
 
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4"])
 def test_low_rank_branch_reduces_error(fmt, tiny):
     """The paper's central claim on a spike + outlier layer: W4A4 with the branch
     beats plain W4A4 on the same smoothed layer, and both beat no smoothing."""
@@ -194,7 +194,7 @@ def test_counting_formulas_eq11_eq12(golden):
 
 # --------------------------------------------------------------- quantized GEMM
 
-@pytest.mark.parametrize("fmt", ["int4", "nvfp4"])
+@pytest.mark.parametrize("fmt", ["int4", "nvfp4", "mxfp4"])
 def test_quantized_gemm_matches_triple_loop(fmt):
     rng = np.random.default_rng(21)
     M, N, K = 6, 5, 128

@@ -255,3 +255,65 @@ def test_pow2_global_scale_boundaries():
         assert O.pow2_global_scale(amax) == 2.0 ** e
         assert O.pow2_global_scale(np.nextafter(amax, 1e30)) == 2.0 ** (e + 1)
         assert O.pow2_global_scale(np.nextafter(amax, 0)) == 2.0 ** e
+
+
+# --------------------------------------------------------------------- MXFP4 g32 (reading 9)
+
+def test_mxfp4_scale_is_the_mx_shared_exponent_and_codes_are_nearest():
+    """X = 2^(floor(log2 amax) - 2) (OCP MX, E2M1 emax = 2), q = nearest E2M1 of x / X."""
+    rng = np.random.default_rng(21)
+    x = O.bf16_rn(rng.standard_normal((40, 256)) * np.exp2(rng.integers(-20, 12, (40, 1))))
+    q = O.quantize_mxfp4_g32(x)
+    a = np.abs(x.reshape(40, 8, 32)).max(-1).astype(np.float64)
+    # floor(log2 a) by brute force over integer exponents: the largest e with 2^e <= a
+    e = np.array([[max(k for k in range(-160, 160) if 2.0 ** k <= v) for v in row] for row in a])
+    assert np.array_equal(q["scale_bits"].astype(np.int64), np.clip(e - 2, -127, 127) + 127)
+    X = np.repeat(2.0 ** (q["scale_bits"].astype(np.int64) - 127), 32, axis=1)
+    v = x.astype(np.float64) / X
+    grid = np.concatenate([-O.E2M1_VALUES[::-1], O.E2M1_VALUES])
+    dv = np.abs(np.minimum(np.abs(v), 6.0)[..., None] - O.E2M1_VALUES)
+    assert np.all(np.abs(np.abs(q["q"]) - np.minimum(np.abs(v), 6.0)) <= dv.min(-1) + 1e-12)
+    assert set(np.unique(q["q"])).issubset(set(grid))
+    # E8M0 byte of the scale, cross-checked with ml_dtypes' float8_e8m0fnu
+    if hasattr(ml_dtypes, "float8_e8m0fnu"):
+        enc = np.asarray(q["scale"][:, :4], np.float32).astype(ml_dtypes.float8_e8m0fnu).view(np.uint8)
+        assert np.array_equal(enc, q["scale_bits"][:, :4])
+
+
+def test_mxfp4_worked_values_and_saturation():
+    g = np.zeros((1, 32), np.float32)
+    # amax 6 * 2^-3: X = 2^-3 and the max element is exactly 6 (code 0x7)
+    g[0, 0] = 0.75
+    g[0, 1] = -0.375                # -3 * 2^-3 -> code 0xD
+    g[0, 2] = 0.03125               # 0.25 * 2^-3: a tie between 0 and 0.5 -> 0 (even)
+    q = O.quantize_mxfp4_g32(g)
+    assert q["scale_bits"][0, 0] == 127 - 3
+    assert (q["codes"][0, 0], q["codes"][0, 1], q["codes"][0, 2]) == (0x7, 0xD, 0x0)
+    # amax 7 * 2^-3: floor(log2) = -1 -> X = 2^-3 and 7 saturates to 6 (the MX conversion clamps)
+    g[0, 0] = 0.875
+    q = O.quantize_mxfp4_g32(g)
+    assert q["scale_bits"][0, 0] == 127 - 3 and q["q"][0, 0] == 6.0
+    # all-zero group: byte 0 (2^-127), zero codes
+    q = O.quantize_mxfp4_g32(np.zeros((2, 64), np.float32))
+    assert np.all(q["scale_bits"] == 0) and np.all(q["codes"] == 0)
+
+
+def test_mxfp4_is_equivariant_under_powers_of_two():
+    rng = np.random.default_rng(22)
+    x = O.bf16_rn(rng.standard_normal((8, 128)))
+    q0 = O.quantize_mxfp4_g32(x)
+    for k in (-9, -1, 3, 17):
+        qk = O.quantize_mxfp4_g32((x * np.float32(2.0 ** k)).astype(np.float32))
+        assert np.array_equal(qk["codes"], q0["codes"])
+        assert np.array_equal(qk["scale_bits"].astype(int), q0["scale_bits"].astype(int) + k)
+
+
+def test_mxfp4_dequant_error_bound():
+    rng = np.random.default_rng(23)
+    x = O.bf16_rn(rng.standard_normal((16, 1024)) * 0.05)
+    q = O.quantize_mxfp4_g32(x)
+    deq = O.dequantize("mxfp4", q)
+    X = np.repeat(q["scale"].astype(np.float64), 32, axis=1)
+    a = np.repeat(np.abs(x.reshape(16, 32, 32)).max(-1), 32, axis=1)
+    # half the largest E2M1 gap (1) times X, plus the clamp of values in (6 X, 8 X)
+    assert np.all(np.abs(x - deq) <= X * 1.0 + np.maximum(a - 6 * X, 0) + 1e-12)
