@@ -46,7 +46,7 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--workload", default="mlp_up")
-    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "int4"])
+    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "int4", "mxfp4"])
     ap.add_argument("--rank", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -92,7 +92,7 @@ def prepare_layer(cfg, fmt, device, weights="svd"):
                 "R_nk": (rng.standard_normal((N, K)) * cfg.sigma_w).astype(np.float32),
                 "L1_rk": (rng.standard_normal((r, K)) * 0.05).astype(np.float32),
                 "L2_nr": (rng.standard_normal((N, r)) * 0.05).astype(np.float32),
-                "act_gscale": P.pow2_tensor_scale(xa) if fmt == "nvfp4" else 1.0}
+                "act_gscale": P.pow2_tensor_scale(xa) if fmt == "nvfp4" else 1.0}   # MXFP4, INT4: none
     packed = P.pack(fmt, prep)
     return layer, prep, packed
 
@@ -494,7 +494,7 @@ def main():
     flops = 2.0 * M * N * K
     value = whole_job_tflops(world, flops, t_step)
     bf16_burst, bf16_sus, hbm, peak_src = peaks()
-    if fmt == "nvfp4":
+    if fmt in ("nvfp4", "mxfp4"):
         peak = bf16_burst * 4.0              # dense FP4 = 4 x dense bf16 (nominal ratio 9 : 2.25)
         peak_note = f"dense FP4 = 4 x {peak_src} bf16 burst"
         src = os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc", "gemm_nvfp4.cu")
@@ -505,8 +505,8 @@ def main():
     alg_flops = flops + 2.0 * M * N * r
     achieved = alg_flops / t_gemm / 1e12
     traffic = recorded_traffic(src, f"{cfg.name}_{fmt}_r{r}")
-    g = 16 if fmt == "nvfp4" else 64
-    sf = 1 if fmt == "nvfp4" else 2
+    g = {"nvfp4": 16, "mxfp4": 32, "int4": 64}[fmt]
+    sf = 2 if fmt == "int4" else 1
     pro_bytes = 2 * M * K + M * K / 2 + M * K / g * sf + 2 * M * r + 2 * r * K + (4 * K)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,

@@ -1,4 +1,11 @@
-// NVFP4 W4A4 GEMM with the fused low-rank up projection (sm_100a, CTA pairs).
+// NVFP4 / MXFP4 W4A4 GEMM with the fused low-rank up projection (sm_100a, CTA pairs).
+//
+// One kernel, two scale flavours: NVFP4 (E4M3 scales per 16 elements, kind::mxf4nvf4
+// block16) and MXFP4 (E8M0 power-of-two scales per 32 elements, kind::mxf4 block32).  The
+// scales of both sit in the same 128-row x 4-group blocked layout; an MXFP4 block covers
+// 128 K elements, so a step carries half as many scale blocks, and each 64-element MMA uses
+// two of the four bytes of a TMEM scale column, picked by the scale-factor id of its
+// instruction descriptor (and the top bits of its scale addresses).
 //
 // "SVDQuant 阅读笔记：用少量高精度计算保护 4-bit 扩散模型", §6.1 "算法 2"
 // steps 4-8 and eq.(7): the 4-bit product Q(X_hat) Q(R) and the 16-bit branch
@@ -46,20 +53,33 @@ constexpr int kEpiWarp0 = 3;
 constexpr int kEpiWarps = 8;
 constexpr uint32_t kABytes = kRows * 128;     // 16 KB
 constexpr uint32_t kBBytes = kRows * 128;     // 16 KB
-constexpr uint32_t kSfaBytes = 2048;          // 128 rows x 16 groups
-constexpr uint32_t kSfbBytes = 4096;          // 256 rows x 16 groups
-constexpr uint32_t kSfaOff = kABytes + kBBytes;
-constexpr uint32_t kSfbOff = kSfaOff + kSfaBytes;
-constexpr uint32_t kStageBytes = kSfbOff + kSfbBytes;   // 38 KB
-constexpr uint32_t kTxMain = 2 * kStageBytes;            // both CTAs
 constexpr uint32_t kTxLowRank = 2 * (kABytes + kBBytes);
+
+// Per-flavour sizes: scale blocks (512 bytes = 128 rows x 4 groups) per step and row block.
+template <bool MX>
+struct Fp4Cfg {
+  static constexpr int kSfBlk = MX ? 2 : 4;                       // 4 groups of 32 or of 16
+  static constexpr uint32_t kSfaBytes = kSfBlk * 512;            // 128 rows
+  static constexpr uint32_t kSfbBytes = 2 * kSfBlk * 512;        // 256 rows (two row blocks)
+  static constexpr uint32_t kSfaOff = kABytes + kBBytes;
+  static constexpr uint32_t kSfbOff = kSfaOff + kSfaBytes;
+  static constexpr uint32_t kStageBytes = kSfbOff + kSfbBytes;   // 38 KB (NVFP4), 35 KB (MXFP4)
+  static constexpr uint32_t kTxMain = 2 * kStageBytes;           // both CTAs
+  static constexpr uint32_t kTmemSfStride = 12 * kSfBlk;         // A-scales 4 cols, B-scales 8 per block
+};
 constexpr uint32_t kEpiBoxBytes = 32 * 128;             // 32 rows x 64 bf16 per epilogue warp
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: accumulator [0, 256); four scale buffers of 48 columns from 256 (A-scales 16,
 // B-scales 32), used round-robin by the main steps.
 constexpr int kSfBufs = 4;
-constexpr uint32_t kTmemSf0 = 256, kTmemSfStride = 48;
+constexpr uint32_t kTmemSf0 = 256;
 
+// E2M1 x E2M1 with UE8M0 scales (bit 23); sf_id (bits 29-30 for A, 4-5 for B) selects the
+// byte of the TMEM scale column where the MMA's scales start.
+__host__ __device__ constexpr uint32_t idesc_mxf4(int m, int n, uint32_t sf_id) {
+  return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(m >> 4) << 24) | (sf_id << 29) | (sf_id << 4);
+}
 __host__ __device__ constexpr uint32_t idesc_nvf4(int m, int n) {
   // E2M1 x E2M1, UE4M3 scales, K-major A and B, dense
   return (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) | (0u << 23) |
@@ -95,11 +115,16 @@ struct SharedTail {
   int abort_flag;
 };
 
+template <bool MX>
 __global__ void __launch_bounds__(kThreads, 1)
-    gemm_nvfp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
+    gemm_fp4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                       const __grid_constant__ CUtensorMap tmap_sfa, const __grid_constant__ CUtensorMap tmap_sfb,
                       const __grid_constant__ CUtensorMap tmap_z, const __grid_constant__ CUtensorMap tmap_l2,
                       const __grid_constant__ CUtensorMap tmap_y, GemmParams p) {
+  using C = Fp4Cfg<MX>;
+  constexpr int kSfBlk = C::kSfBlk;
+  constexpr uint32_t kSfaOff = C::kSfaOff, kSfbOff = C::kSfbOff, kStageBytes = C::kStageBytes;
+  constexpr uint32_t kTxMain = C::kTxMain, kTmemSfStride = C::kTmemSfStride;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* epi_smem = smem + kStages * kStageBytes;                       // 8 x 4 KB staging for Y
@@ -168,8 +193,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], kTxMain);
             ptx::tma_load_2d_pair(st, &tmap_a, full_leader, k * (kKTile / 2), m0);
             ptx::tma_load_2d_pair(st + kABytes, &tmap_b, full_leader, k * (kKTile / 2), nb0);
-            ptx::tma_load_3d_pair(st + kSfaOff, &tmap_sfa, full_leader, 0, k * (kKTile / 64), m0 / 128);
-            ptx::tma_load_3d_pair(st + kSfbOff, &tmap_sfb, full_leader, 0, k * (kKTile / 64), n0 / 128);
+            ptx::tma_load_3d_pair(st + kSfaOff, &tmap_sfa, full_leader, 0, k * kSfBlk, m0 / 128);
+            ptx::tma_load_3d_pair(st + kSfbOff, &tmap_sfb, full_leader, 0, k * kSfBlk, n0 / 128);
           } else {
             const int c = k - nk_main;
             if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], kTxLowRank);
@@ -202,12 +227,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) {
             const uint32_t st = ptx::smem_u32(smem + s * kStageBytes);
             const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
+            const int nblk = MX ? (nkb + 1) / 2 : nkb;            // scale blocks of this step
             const uint32_t sfa = tmem + kTmemSf0 + b * kTmemSfStride;
-            const uint32_t sfb = sfa + 16;
-            for (int kb = 0; kb < nkb; ++kb) {
-              ptx::tmem_cp_32x128b_warpx4_pair(sfa + kb * 4, ptx::sdesc_sf(st + kSfaOff + kb * 512));
-              ptx::tmem_cp_32x128b_warpx4_pair(sfb + kb * 8, ptx::sdesc_sf(st + kSfbOff + kb * 512));
-              ptx::tmem_cp_32x128b_warpx4_pair(sfb + kb * 8 + 4, ptx::sdesc_sf(st + kSfbOff + 2048 + kb * 512));
+            const uint32_t sfb = sfa + 4 * kSfBlk;
+            for (int blk = 0; blk < nblk; ++blk) {
+              ptx::tmem_cp_32x128b_warpx4_pair(sfa + blk * 4, ptx::sdesc_sf(st + kSfaOff + blk * 512));
+              ptx::tmem_cp_32x128b_warpx4_pair(sfb + blk * 8, ptx::sdesc_sf(st + kSfbOff + blk * 512));
+              ptx::tmem_cp_32x128b_warpx4_pair(sfb + blk * 8 + 4,
+                                               ptx::sdesc_sf(st + kSfbOff + kSfBlk * 512 + blk * 512));
             }
             ptx::tc_commit_pair_local(&sh->sf_ready[b]);
           }
@@ -243,10 +270,18 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (main_step) {
               const int nkb = min(kKTile / 64, kblk64 - k * (kKTile / 64));
               const uint32_t sfa = tmem + kTmemSf0 + b * kTmemSfStride;
-              const uint32_t sfb = sfa + 16;
+              const uint32_t sfb = sfa + 4 * kSfBlk;
               for (int kb = 0; kb < nkb; ++kb) {
-                ptx::umma_nvf4_pair(tmem, ptx::sdesc_sw128(st + kb * 32), ptx::sdesc_sw128(st + kABytes + kb * 32),
-                                    id4, sfa + kb * 4, sfb + kb * 8, (k | kb) != 0 ? 1u : 0u);
+                const uint64_t adesc = ptx::sdesc_sw128(st + kb * 32), bdesc = ptx::sdesc_sw128(st + kABytes + kb * 32);
+                const uint32_t acc = (k | kb) != 0 ? 1u : 0u;
+                if (MX) {
+                  // block kb/2 of 4 scales per row; this MMA's two start at byte 2 (kb & 1)
+                  const uint32_t id = (kb & 1) * 2u;
+                  ptx::umma_mxf4_pair(tmem, adesc, bdesc, idesc_mxf4(kBM, kBN, id), (sfa + (kb >> 1) * 4) | (id << 30),
+                                      (sfb + (kb >> 1) * 8) | (id << 30), acc);
+                } else {
+                  ptx::umma_nvf4_pair(tmem, adesc, bdesc, id4, sfa + kb * 4, sfb + kb * 8, acc);
+                }
               }
               ptx::tc_commit_pair_local(&sh->sf_free[b]);
             } else {
@@ -348,6 +383,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+template <bool MX>
 int max_active_clusters(size_t smem) {
   static int cache[64] = {0};
   int dev = 0;
@@ -365,7 +401,7 @@ int max_active_clusters(size_t smem) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, gemm_nvfp4_kernel, &cfg) != cudaSuccess || n <= 0) {
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_fp4_kernel<MX>, &cfg) != cudaSuccess || n <= 0) {
     cudaGetLastError();
     return 0;
   }
@@ -373,18 +409,20 @@ int max_active_clusters(size_t smem) {
   return n;
 }
 
-}  // namespace
+template <bool MX>
+size_t smem_bytes() {
+  return 1024 + kStages * Fp4Cfg<MX>::kStageBytes + kEpiWarps * kEpiBoxBytes + sizeof(SharedTail);
+}
 
-size_t gemm_nvfp4_smem_bytes() { return 1024 + kStages * kStageBytes + kEpiWarps * kEpiBoxBytes + sizeof(SharedTail); }
-
-cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
-                              const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
-                              const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s) {
-  const size_t smem = gemm_nvfp4_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_nvfp4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+template <bool MX>
+cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa, const CUtensorMap& tsfb,
+                   const CUtensorMap& tz, const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p,
+                   int num_sms, cudaStream_t s) {
+  const size_t smem = smem_bytes<MX>();
+  cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  int clusters = max_active_clusters(smem);
+  int clusters = max_active_clusters<MX>(smem);
   if (clusters <= 0) clusters = num_sms / 2;
   if (clusters > p.num_tiles) clusters = p.num_tiles;
   cudaLaunchConfig_t cfg = {};
@@ -399,9 +437,18 @@ cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, cons
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_nvfp4_kernel, ta, tb, tsfa, tsfb, tz, tl2, ty, p);
+  e = cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<MX>, ta, tb, tsfa, tsfb, tz, tl2, ty, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+}  // namespace
+
+cudaError_t launch_gemm_fp4(bool mx, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
+                            const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
+                            const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s) {
+  return mx ? launch<true>(ta, tb, tsfa, tsfb, tz, tl2, ty, p, num_sms, s)
+            : launch<false>(ta, tb, tsfa, tsfb, tz, tl2, ty, p, num_sms, s);
 }
 
 }  // namespace svdq

@@ -7,6 +7,7 @@
 // NVFP4 groups of 16 with an FP8 (E4M3) scale.  The rounding rules are the
 // ones stated in svdq.h; every conversion below is written from the format
 // definition (IEEE binary16, bfloat16, OCP E4M3 "fn", E2M1).
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <cstring>
@@ -127,8 +128,8 @@ bool is_pow2_positive(float g) {
   return m == 0.5f;
 }
 
-size_t nvfp4_sf_offset(int64_t row, int64_t grp, int64_t K) {
-  return static_cast<size_t>(((row / 128) * (K / 64) + grp / 4) * 512 + (row % 32) * 16 +
+size_t blocked_sf_offset(int64_t row, int64_t grp, int64_t K, int g) {
+  return static_cast<size_t>(((row / 128) * (K / (4 * g)) + grp / 4) * 512 + (row % 32) * 16 +
                              ((row % 128) / 32) * 4 + (grp % 4));
 }
 
@@ -145,7 +146,7 @@ extern "C" svdq_status svdq_pack_weight(svdq_format fmt, int64_t N, int64_t K, i
   if (!R || !w_codes || !w_scales || !w_gscale) return SVDQ_ERR_INVALID_ARG;
   if (rank > 0 && (!L1 || !L2 || !L1_bf16 || !L2_bf16)) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_positive(act_gscale)) return SVDQ_ERR_INVALID_ARG;
-  if (fmt == SVDQ_FMT_INT4_G64 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_FMT_NVFP4_G16 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
 
   uint8_t* codes = static_cast<uint8_t*>(w_codes);
   std::memset(codes, 0, static_cast<size_t>(N) * static_cast<size_t>(K / 2));
@@ -165,12 +166,35 @@ extern "C" svdq_status svdq_pack_weight(svdq_format fmt, int64_t N, int64_t K, i
         for (int j = 0; j < 16; ++j) a = std::fmax(a, std::fabs(row[g * 16 + j]));
         float t = (a / 6.0f) / gw;
         uint8_t sc = f32_to_e4m3_rn_sat(t);
-        sf[nvfp4_sf_offset(n, g, K)] = sc;
+        sf[blocked_sf_offset(n, g, K, 16)] = sc;
         float den = e4m3_to_f32(sc) * gw;
         for (int j = 0; j < 16; ++j) {
           int64_t k = g * 16 + j;
           uint8_t c = 0;
           if (den > 0.0f) c = f32_to_e2m1_rn_sat(row[k] / den);
+          codes[n * (K / 2) + k / 2] |= static_cast<uint8_t>((k & 1) ? (c << 4) : c);
+        }
+      }
+    }
+  } else if (fmt == SVDQ_FMT_MXFP4_G32) {
+    // MX shared scale: X = 2^clamp(floor(log2 a) - 2, -127, 127), byte log2(X) + 127
+    uint8_t* sf = static_cast<uint8_t*>(w_scales);
+    std::memset(sf, 0, static_cast<size_t>(Np) * static_cast<size_t>(K / 32));
+    for (int64_t n = 0; n < N; ++n) {
+      const float* row = R + n * K;
+      for (int64_t g = 0; g < K / 32; ++g) {
+        float a = 0.0f;
+        for (int j = 0; j < 32; ++j) a = std::fmax(a, std::fabs(row[g * 32 + j]));
+        int e = -127;
+        if (a > 0.0f) {
+          int ex = 0;
+          std::frexp(a, &ex);            // a = m 2^ex, m in [0.5, 1): floor(log2 a) = ex - 1
+          e = std::min(127, std::max(-127, ex - 1 - 2));
+        }
+        sf[blocked_sf_offset(n, g, K, 32)] = static_cast<uint8_t>(e + 127);
+        for (int j = 0; j < 32; ++j) {
+          const int64_t k = g * 32 + j;
+          const uint8_t c = f32_to_e2m1_rn_sat(std::ldexp(row[k], -e));   // exact: x / 2^e
           codes[n * (K / 2) + k / 2] |= static_cast<uint8_t>((k & 1) ? (c << 4) : c);
         }
       }

@@ -294,7 +294,53 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
             sc_pack_b |= (sab >> 8) << (8 * j);
           }
         }
-        if (FMT == kFmtInt4) {
+        if (FMT == kFmtMxfp4) {
+          // two 32-element groups per row per box (k16 tiles 0-1 and 2-3).  X = 2^s with
+          // s = clamp(floor(log2 a) - 2, -127, 127): for a normal absmax a the exponent field f
+          // gives the E8M0 byte max(f - 2, 0); zero and subnormal a give byte 0 (s = -127).
+          uint32_t sb_a = 0, sb_b = 0;
+#pragma unroll
+          for (int gi = 0; gi < 2; ++gi) {
+            const int j0 = 2 * gi;
+            float ma = fmaxf(fmaxf(fmaxf(fabsf(nx[j0][0].x), fabsf(nx[j0][0].y)), fmaxf(fabsf(nx[j0][1].x), fabsf(nx[j0][1].y))),
+                             fmaxf(fmaxf(fabsf(nx[j0 + 1][0].x), fabsf(nx[j0 + 1][0].y)), fmaxf(fabsf(nx[j0 + 1][1].x), fabsf(nx[j0 + 1][1].y))));
+            float mb = fmaxf(fmaxf(fmaxf(fabsf(nx[j0][2].x), fabsf(nx[j0][2].y)), fmaxf(fabsf(nx[j0][3].x), fabsf(nx[j0][3].y))),
+                             fmaxf(fmaxf(fabsf(nx[j0 + 1][2].x), fabsf(nx[j0 + 1][2].y)), fmaxf(fabsf(nx[j0 + 1][3].x), fabsf(nx[j0 + 1][3].y))));
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 1));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 1));
+            ma = fmaxf(ma, __shfl_xor_sync(0xffffffffu, ma, 2));
+            mb = fmaxf(mb, __shfl_xor_sync(0xffffffffu, mb, 2));
+            const int fa = static_cast<int>(__float_as_uint(ma) >> 23);    // |a|: sign bit is 0
+            const int fb = static_cast<int>(__float_as_uint(mb) >> 23);
+            const uint32_t ba = static_cast<uint32_t>(max(fa - 2, 0)), bb = static_cast<uint32_t>(max(fb - 2, 0));
+            sb_a |= ba << (8 * gi);
+            sb_b |= bb << (8 * gi);
+            // -1/X = -2^(127 - byte): exponent field 254 - byte (2..254, always normal); the
+            // product with -x_hat is x_hat / X exactly
+            const float na = -__uint_as_float((254u - ba) << 23), nb = -__uint_as_float((254u - bb) << 23);
+            const float2 naa = make_float2(na, na), nbb = make_float2(nb, nb);
+#pragma unroll
+            for (int jj = j0; jj < j0 + 2; ++jj) {
+              const float2 q0 = __fmul2_rn(nx[jj][0], naa), q1 = __fmul2_rn(nx[jj][1], naa);
+              const float2 q2 = __fmul2_rn(nx[jj][2], nbb), q3 = __fmul2_rn(nx[jj][3], nbb);
+              cst[g * 32 + jj * 8 + tig] = static_cast<uint8_t>(ptx::cvt_e2m1x2(q0.x, q0.y));
+              cst[g * 32 + jj * 8 + 4 + tig] = static_cast<uint8_t>(ptx::cvt_e2m1x2(q1.x, q1.y));
+              cst[(g + 8) * 32 + jj * 8 + tig] = static_cast<uint8_t>(ptx::cvt_e2m1x2(q2.x, q2.y));
+              cst[(g + 8) * 32 + jj * 8 + 4 + tig] = static_cast<uint8_t>(ptx::cvt_e2m1x2(q3.x, q3.y));
+            }
+          }
+          if (tig == 0) {
+            // two consecutive E8M0 bytes of the 128x4 blocked layout (groups of 32) per row
+            const int grp = col0 / 32;               // first of the box's two groups
+            uint8_t* sc = reinterpret_cast<uint8_t*>(p.scales);
+            const size_t ba = (static_cast<size_t>(row_a / 128) * (p.K / 128) + grp / 4) * 512 +
+                              (row_a % 32) * 16 + ((row_a % 128) / 32) * 4 + grp % 4;
+            const size_t bb = (static_cast<size_t>(row_b / 128) * (p.K / 128) + grp / 4) * 512 +
+                              (row_b % 32) * 16 + ((row_b % 128) / 32) * 4 + grp % 4;
+            *reinterpret_cast<uint16_t*>(sc + ba) = static_cast<uint16_t>(sb_a);
+            *reinterpret_cast<uint16_t*>(sc + bb) = static_cast<uint16_t>(sb_b);
+          }
+        } else if (FMT == kFmtInt4) {
           // one 64-element group per row per box
           float ma = 0.f, mb = 0.f;
 #pragma unroll
@@ -455,7 +501,9 @@ static cudaError_t launch_pro_rank(const CUtensorMap& tx, const CUtensorMap& tl1
 
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
                             cudaStream_t s) {
-  return fmt == kFmtNvfp4 ? launch_pro_rank<kFmtNvfp4>(tx, tl1, p, s) : launch_pro_rank<kFmtInt4>(tx, tl1, p, s);
+  if (fmt == kFmtNvfp4) return launch_pro_rank<kFmtNvfp4>(tx, tl1, p, s);
+  if (fmt == kFmtMxfp4) return launch_pro_rank<kFmtMxfp4>(tx, tl1, p, s);
+  return launch_pro_rank<kFmtInt4>(tx, tl1, p, s);
 }
 
 }  // namespace svdq

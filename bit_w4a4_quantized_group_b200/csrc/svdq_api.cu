@@ -70,11 +70,12 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint
   return r == CUDA_SUCCESS;
 }
 
-// The 128x4 blocked E4M3 scale layout seen as [rows/128][K/64][64 x 8-byte words]:
-// one TMA box = `blocks` row blocks x 4 groups-of-4 = the scales of 128*blocks rows x 256 columns.
-bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows_pad, int64_t K, uint32_t blocks) {
-  return make_tmap_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT64, 64, static_cast<uint64_t>(K / 64),
-                      static_cast<uint64_t>(rows_pad / 128), 512, static_cast<uint64_t>(K / 64) * 512, 64, 4, blocks);
+// The 128x4 blocked scale layout (groups of g) seen as [rows/128][K/(4g)][64 x 8-byte words]:
+// one TMA box = `blocks` row blocks x the scale blocks of 256 columns (4 for g = 16, 2 for g = 32).
+bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows_pad, int64_t K, int g, uint32_t blocks) {
+  const uint64_t kblocks = static_cast<uint64_t>(K / (4 * g));
+  return make_tmap_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT64, 64, kblocks, static_cast<uint64_t>(rows_pad / 128), 512,
+                      kblocks * 512, 64, static_cast<uint32_t>(256 / (4 * g)), blocks);
 }
 
 int device_sm_count() {
@@ -98,7 +99,8 @@ int* device_error_word() {
 
 size_t scale_bytes(svdq_format fmt, int64_t rows, int64_t K) {
   const int64_t rp = (rows + 127) / 128 * 128;
-  return fmt == SVDQ_FMT_NVFP4_G16 ? static_cast<size_t>(rp * (K / 16)) : static_cast<size_t>(rp * (K / 64) * 2);
+  if (fmt == SVDQ_FMT_INT4_G64) return static_cast<size_t>(rp * (K / 64) * 2);
+  return static_cast<size_t>(rp * (K / fp4_group(fmt)));
 }
 
 }  // namespace
@@ -179,7 +181,7 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   if (lambda && !aligned16(lambda)) return SVDQ_ERR_INVALID_ARG;
   if (rank > 0 && (!L1_bf16 || !Z_bf16 || !aligned16(L1_bf16) || !aligned16(Z_bf16))) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_positive(act_gscale)) return SVDQ_ERR_INVALID_ARG;
-  if (fmt == SVDQ_FMT_INT4_G64 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_FMT_NVFP4_G16 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
 
   // X and L1 seen as [K/64 column blocks][rows][64 columns]: one load brings kProBoxes
   // 64-column boxes (128B-swizzled) of 32 X rows or of all L1 rows
@@ -207,7 +209,8 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   p.Z = static_cast<__nv_bfloat16*>(Z_bf16);
   p.err = device_error_word();
   if (!p.err) return SVDQ_ERR_CUDA;
-  cudaError_t e = launch_prologue(fmt == SVDQ_FMT_NVFP4_G16 ? kFmtNvfp4 : kFmtInt4, tx, tl1, p,
+  const int kf = fmt == SVDQ_FMT_NVFP4_G16 ? kFmtNvfp4 : (fmt == SVDQ_FMT_MXFP4_G32 ? kFmtMxfp4 : kFmtInt4);
+  cudaError_t e = launch_prologue(kf, tx, tl1, p,
                                   static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return cuda_fail(e);
   t_last_launch_count = 1;
@@ -229,7 +232,7 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
   if (bias_bf16 && !aligned16(bias_bf16)) return SVDQ_ERR_INVALID_ARG;
   if (rank > 0 && (!Z_bf16 || !L2_bf16 || !aligned16(Z_bf16) || !aligned16(L2_bf16))) return SVDQ_ERR_INVALID_ARG;
   if (!is_pow2_positive(act_gscale) || !is_pow2_positive(w_gscale)) return SVDQ_ERR_INVALID_ARG;
-  if (fmt == SVDQ_FMT_INT4_G64 && (act_gscale != 1.0f || w_gscale != 1.0f)) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_FMT_NVFP4_G16 && (act_gscale != 1.0f || w_gscale != 1.0f)) return SVDQ_ERR_INVALID_ARG;
 
   const int sms = device_sm_count();
   if (sms <= 0) return SVDQ_ERR_CUDA;
@@ -252,15 +255,16 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
 
   CUtensorMap tz, tl2;
   cudaError_t e;
-  if (fmt == SVDQ_FMT_NVFP4_G16) {
+  if (fmt == SVDQ_FMT_NVFP4_G16 || fmt == SVDQ_FMT_MXFP4_G32) {
+    const int g = fp4_group(fmt);
     p.tiles_m = static_cast<int>((M + 255) / 256);
     p.tiles_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.tiles_m * p.tiles_n;
     CUtensorMap ta, tb, tsfa, tsfb;
     if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) return SVDQ_ERR_CUDA;
     if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) return SVDQ_ERR_CUDA;
-    if (!make_tmap_sf(&tsfa, a_scales, p.Mpad, K, 1)) return SVDQ_ERR_CUDA;
-    if (!make_tmap_sf(&tsfb, w_scales, p.Npad, K, 2)) return SVDQ_ERR_CUDA;
+    if (!make_tmap_sf(&tsfa, a_scales, p.Mpad, K, g, 1)) return SVDQ_ERR_CUDA;
+    if (!make_tmap_sf(&tsfb, w_scales, p.Npad, K, g, 2)) return SVDQ_ERR_CUDA;
     if (rank > 0) {
       if (!make_tmap(&tz, Z_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, M, 64, 128)) return SVDQ_ERR_CUDA;
       if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 128)) return SVDQ_ERR_CUDA;
@@ -270,7 +274,8 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
     }
     CUtensorMap ty;
     if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
-    e = launch_gemm_nvfp4(ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms, static_cast<cudaStream_t>(cuda_stream));
+    e = launch_gemm_fp4(fmt == SVDQ_FMT_MXFP4_G32, ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms,
+                        static_cast<cudaStream_t>(cuda_stream));
   } else {
     p.tiles_m = static_cast<int>((M + 127) / 128);
     p.tiles_n = static_cast<int>(N / 128);

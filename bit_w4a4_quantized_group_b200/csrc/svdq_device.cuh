@@ -11,6 +11,7 @@ namespace svdq {
 
 constexpr int kFmtNvfp4 = 1;
 constexpr int kFmtInt4 = 2;
+constexpr int kFmtMxfp4 = 3;
 
 // Codes recorded in the device error word when a bounded wait runs out.
 enum : int {
@@ -90,10 +91,10 @@ struct GemmParams {
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
                             cudaStream_t s);
 
-size_t gemm_nvfp4_smem_bytes();
-cudaError_t launch_gemm_nvfp4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
-                              const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
-                              const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
+// NVFP4 (mx = false) or MXFP4 (mx = true) GEMM with the fused low-rank up projection.
+cudaError_t launch_gemm_fp4(bool mx, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
+                            const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
+                            const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
 size_t gemm_int4_smem_bytes();
 cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
                              const CUtensorMap& tl2, const CUtensorMap& ty, const CUtensorMap& tsa,

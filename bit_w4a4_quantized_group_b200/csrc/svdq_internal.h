@@ -11,7 +11,7 @@ namespace svdq {
 constexpr int kMaxRank = 128;
 
 inline svdq_status check_dims(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank) {
-  if (fmt != SVDQ_FMT_NVFP4_G16 && fmt != SVDQ_FMT_INT4_G64) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_FMT_NVFP4_G16 && fmt != SVDQ_FMT_INT4_G64 && fmt != SVDQ_FMT_MXFP4_G32) return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || N < 128 || K < 128) return SVDQ_ERR_INVALID_ARG;
   if (K % 128 != 0 || N % 128 != 0) return SVDQ_ERR_INVALID_ARG;
   if (rank < 0 || rank > kMaxRank || rank % 16 != 0) return SVDQ_ERR_INVALID_ARG;
@@ -32,6 +32,9 @@ float e4m3_to_f32(uint8_t c);
 uint8_t f32_to_e2m1_rn_sat(float v);
 float pow2_gscale(float amax);
 bool is_pow2_positive(float g);
-size_t nvfp4_sf_offset(int64_t row, int64_t grp, int64_t K);
+// Byte offset of the scale of (row, group) in the 128x4 blocked layout, groups of g elements.
+size_t blocked_sf_offset(int64_t row, int64_t grp, int64_t K, int g);
+// Group size of an E2M1 format (16 NVFP4, 32 MXFP4).
+inline int fp4_group(svdq_format fmt) { return fmt == SVDQ_FMT_MXFP4_G32 ? 32 : 16; }
 
 }  // namespace svdq

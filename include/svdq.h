@@ -15,7 +15,7 @@
  * already-decomposed layer.
  *
  * Notation: M = tokens (b), K = input features (m), N = output features (n),
- * r = rank of the low-rank branch.  g = 16 (NVFP4) or 64 (INT4), G = K / g.
+ * r = rank of the low-rank branch.  g = 16 (NVFP4), 32 (MXFP4) or 64 (INT4), G = K / g.
  *
  * Conventions for every call
  *   - Ownership: the caller owns every buffer.  The library never allocates
@@ -44,12 +44,13 @@
  *   Y        bf16 [M][N]
  *   codes    u8   [rows][K/2]            element k of a row in the low nibble of
  *                                        byte k/2 when k is even, high nibble when odd.
- *                                        NVFP4: E2M1 code (bit 3 = sign);
+ *                                        NVFP4, MXFP4: E2M1 code (bit 3 = sign);
  *                                        INT4: 4-bit two's complement in -7..7.
- *   NVFP4 scales  u8 (E4M3), "128x4 blocked" layout, rows padded to Rp = ceil(rows/128)*128:
- *       byte offset of (row, grp) = ((row/128)*(K/64) + grp/4)*512
+ *   NVFP4 scales  u8 (E4M3), MXFP4 scales u8 (E8M0: the scale is 2^(byte - 127)), both in the
+ *       "128x4 blocked" layout, rows padded to Rp = ceil(rows/128)*128:
+ *       byte offset of (row, grp) = ((row/128)*(K/(4g)) + grp/4)*512
  *                                   + (row%32)*16 + ((row%128)/32)*4 + grp%4
- *       size = Rp * K / 16 bytes.  Padding rows hold 0.
+ *       size = Rp * K / g bytes.  Padding rows hold 0.
  *   INT4 scales   fp16, group-major, rows padded to Rp = ceil(rows/128)*128:
  *       element offset of (row, grp) = grp*Rp + row;  size = Rp * (K/64) * 2 bytes.
  *   ("rows" is M for activations, N for weights.)
@@ -78,7 +79,14 @@ typedef enum {
   SVDQ_FMT_NVFP4_G16 = 1,
   /* symmetric INT4 codes -7..7, groups of 64 along K, fp16 group scales
    * ("SVDQuant 阅读笔记" §2.2 eq.(1) and §8: INT4 g64 with 16-bit scale). */
-  SVDQ_FMT_INT4_G64 = 2
+  SVDQ_FMT_INT4_G64 = 2,
+  /* E2M1 codes, groups of 32 along K, one shared power-of-two scale per group stored
+   * as its E8M0 byte: X = 2^(floor(log2 a) - 2), clamped to [2^-127, 2^127], the MX
+   * shared scale of the OCP Microscaling format for E2M1 (largest value 6 = 1.5 * 2^2);
+   * q = e2m1_satfinite(x / X).  No tensor scale: act_gscale and w_gscale are 1.
+   * ("SVDQuant（实验性功能）": the Nunchaku export uses MXFP4 E2M1 W4A4, group size 32,
+   * symmetric.) */
+  SVDQ_FMT_MXFP4_G32 = 3
 } svdq_format;
 
 /* Byte sizes of every buffer of one layer call (no allocation happens). */
@@ -112,12 +120,13 @@ svdq_status svdq_buffer_sizes(svdq_format fmt, int64_t M, int64_t N, int64_t K, 
  *                       NVFP4: s = e4m3_satfinite(fp32(fp32(a/6)/g_w)),
  *                              q = e2m1_satfinite(fp32(x/(s*g_w)))
  *                       with a = max|x| over the group (a zero scale gives zero codes)
+ *                       MXFP4: the rule of SVDQ_FMT_MXFP4_G32 (a zero group gets byte 0)
  *   *w_gscale           NVFP4: g_w = 2^ceil(log2(max|R| / (6*448))) (1 if R == 0);
- *                       INT4: 1
+ *                       INT4, MXFP4: 1
  *   L1_bf16             bf16 of L1 (round to nearest even)
  *   L2_bf16             bf16 of bf16(L2) / (act_gscale * g_w); must be exact
  * act_gscale is the activation tensor scale later given to the device calls
- * (a positive power of two; use 1 for INT4).  Returns SVDQ_ERR_INVALID_ARG for
+ * (a positive power of two; 1 for INT4 and MXFP4).  Returns SVDQ_ERR_INVALID_ARG for
  * bad sizes / NULL pointers / a non power-of-two act_gscale, and
  * SVDQ_ERR_UNSUPPORTED if pre-dividing L2 would not be exact in bf16.
  */
@@ -130,7 +139,7 @@ svdq_status svdq_pack_weight(svdq_format fmt, int64_t N, int64_t K, int rank, fl
  * Device prologue ("算法 2" steps 1-3 of "SVDQuant 阅读笔记" §6.1): one read of X.
  *   X_hat = bf16(fp32(X) / lambda)            (IEEE fp32 divide, one bf16 rounding)
  *   a_codes, a_scales = group quantization of X_hat along K (rules of svdq_pack_weight,
- *                       with act_gscale in place of g_w; INT4 requires act_gscale == 1)
+ *                       with act_gscale in place of g_w; INT4 and MXFP4 require act_gscale == 1)
  *   Z = bf16(X_hat L1^T)                      (fp32 accumulation; skipped when rank == 0)
  * X, lambda, L1 are inputs; a_codes, a_scales, Z outputs (Z may be NULL when rank == 0).
  */

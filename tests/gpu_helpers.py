@@ -5,7 +5,7 @@ import torch
 
 from bit_w4a4_quantized_group_b200 import binding as B
 
-from layouts import (bf16_bits_to_f32, f32_to_bf16_bits_exact, nvfp4_scale_offsets, scales_canonical,
+from layouts import (bf16_bits_to_f32, blocked_scale_offsets, f32_to_bf16_bits_exact, scales_canonical,
                      scales_padding, unpack_codes)
 
 
@@ -50,9 +50,10 @@ def run_prologue(fmt, X, lam, gx, L1_rk, fill=0x5A):
 def encode_scales(fmt, scale_bits: np.ndarray, rows: int, K: int) -> np.ndarray:
     """Canonical scale bits [rows][G] -> library buffer bytes (padding rows zero)."""
     rp = (rows + 127) // 128 * 128
-    if fmt == "nvfp4":
-        buf = np.zeros(rp * K // 16, np.uint8)
-        buf[nvfp4_scale_offsets(rows, K)] = scale_bits
+    if fmt in ("nvfp4", "mxfp4"):
+        g = 16 if fmt == "nvfp4" else 32
+        buf = np.zeros(rp * K // g, np.uint8)
+        buf[blocked_scale_offsets(rows, K, g)] = scale_bits
         return buf
     buf = np.zeros((K // 64, rp), np.uint16)
     buf[:, :rows] = scale_bits.T

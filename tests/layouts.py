@@ -20,26 +20,38 @@ def pack_codes(codes: np.ndarray) -> np.ndarray:
     return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8)
 
 
-def nvfp4_scale_offsets(rows: int, K: int) -> np.ndarray:
-    """Byte offset of (row, group) in the 128x4 blocked E4M3 scale layout."""
+def blocked_scale_offsets(rows: int, K: int, g: int = 16) -> np.ndarray:
+    """Byte offset of (row, group) in the 128x4 blocked scale layout, groups of g elements."""
     r = np.arange(rows)[:, None]
-    g = np.arange(K // 16)[None, :]
-    return ((r // 128) * (K // 64) + g // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + g % 4
+    grp = np.arange(K // g)[None, :]
+    return ((r // 128) * (K // (4 * g)) + grp // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + grp % 4
+
+
+def nvfp4_scale_offsets(rows: int, K: int) -> np.ndarray:
+    return blocked_scale_offsets(rows, K, 16)
+
+
+def blocked_scales_canonical(buf: np.ndarray, rows: int, K: int, g: int = 16) -> np.ndarray:
+    b = np.asarray(buf, np.uint8).reshape(-1)
+    return b[blocked_scale_offsets(rows, K, g)]
 
 
 def nvfp4_scales_canonical(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
-    b = np.asarray(buf, np.uint8).reshape(-1)
-    return b[nvfp4_scale_offsets(rows, K)]
+    return blocked_scales_canonical(buf, rows, K, 16)
 
 
-def nvfp4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+def blocked_scales_padding(buf: np.ndarray, rows: int, K: int, g: int = 16) -> np.ndarray:
     """Bytes of the padding rows (rows .. ceil(rows/128)*128 - 1)."""
     rp = (rows + 127) // 128 * 128
     if rp == rows:
         return np.zeros(0, np.uint8)
     b = np.asarray(buf, np.uint8).reshape(-1)
-    off = nvfp4_scale_offsets(rp, K)[rows:]
+    off = blocked_scale_offsets(rp, K, g)[rows:]
     return b[off]
+
+
+def nvfp4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
+    return blocked_scales_padding(buf, rows, K, 16)
 
 
 def int4_scales_canonical(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
@@ -56,11 +68,15 @@ def int4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
 
 
 def scales_canonical(fmt: str, buf, rows: int, K: int) -> np.ndarray:
-    return nvfp4_scales_canonical(buf, rows, K) if fmt == "nvfp4" else int4_scales_canonical(buf, rows, K)
+    if fmt == "int4":
+        return int4_scales_canonical(buf, rows, K)
+    return blocked_scales_canonical(buf, rows, K, 16 if fmt == "nvfp4" else 32)
 
 
 def scales_padding(fmt: str, buf, rows: int, K: int) -> np.ndarray:
-    return nvfp4_scales_padding(buf, rows, K) if fmt == "nvfp4" else int4_scales_padding(buf, rows, K)
+    if fmt == "int4":
+        return int4_scales_padding(buf, rows, K)
+    return blocked_scales_padding(buf, rows, K, 16 if fmt == "nvfp4" else 32)
 
 
 def bf16_bits_to_f32(bits: np.ndarray) -> np.ndarray:

@@ -16,7 +16,7 @@ from bit_w4a4_quantized_group_b200 import binding as B
 from bit_w4a4_quantized_group_b200 import build as BUILD
 from bit_w4a4_quantized_group_b200 import inputs as I
 
-from layouts import int4_scales_canonical, nvfp4_scales_canonical, scales_padding, unpack_codes
+from layouts import int4_scales_canonical, nvfp4_scales_canonical, scales_canonical, scales_padding, unpack_codes
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -121,10 +121,7 @@ def _check_pack(fmt, R_nk, L1_rk, L2_nr, gx):
     ref = O.pack_weight(fmt, R_nk, L1_rk, L2_nr, gx)
     assert got["w_gscale"] == ref["gscale"]
     assert np.array_equal(unpack_codes(got["w_codes"], N, K), ref["q"]["codes"])
-    if fmt == "nvfp4":
-        assert np.array_equal(nvfp4_scales_canonical(got["w_scales"], N, K), ref["q"]["scale_bits"])
-    else:
-        assert np.array_equal(int4_scales_canonical(got["w_scales"], N, K), ref["q"]["scale_bits"])
+    assert np.array_equal(scales_canonical(fmt, got["w_scales"], N, K), ref["q"]["scale_bits"])
     assert np.all(scales_padding(fmt, got["w_scales"], N, K) == 0)
     if L1_rk is not None and L1_rk.shape[0] > 0:
         l1 = (got["L1_bf16"].astype(np.uint32) << 16).view(np.float32)
@@ -133,7 +130,7 @@ def _check_pack(fmt, R_nk, L1_rk, L2_nr, gx):
         assert np.array_equal(l2, ref["L2_scaled"])
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 def test_pack_weight_matches_reference_on_tiny_layer(lib, fmt):
     layer = I.make_layer(I.TINY)
     prep = O.prepare_layer(fmt, layer.X, layer.W, 16)
@@ -141,7 +138,7 @@ def test_pack_weight_matches_reference_on_tiny_layer(lib, fmt):
                 prep["act_gscale"])
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 @pytest.mark.parametrize("scale_exp", [-12, -3, 0, 6])
 def test_pack_weight_matches_reference_random(lib, fmt, scale_exp):
     rng = np.random.default_rng(100 + scale_exp)
@@ -169,6 +166,14 @@ def test_pack_weight_rank0_and_ties(lib):
     R2[:, 0] = 7.0
     R2[:, 1:6] = [0.5, 1.5, 2.5, -0.5, -3.5]
     _check_pack("int4", R2, None, None, 1.0)
+    # MXFP4: amax 6 gives X = 1 and the same E2M1 midpoints; amax 7 saturates; a tiny group
+    _check_pack("mxfp4", R, None, None, 1.0)
+    R3 = np.zeros((N, K), np.float32)
+    R3[:, 0] = 7.0
+    R3[:, 1:5] = [0.25, -0.75, 3.5, 5.0]
+    R3[:, 32] = 2.0 ** -140
+    R3[:, 64] = -0.0
+    _check_pack("mxfp4", R3, None, None, 1.0)
 
 
 def test_pack_weight_rejects(lib):
@@ -178,6 +183,8 @@ def test_pack_weight_rejects(lib):
         B.pack_weight_np("nvfp4", R, None, None, 3.0)     # not a power of two
     with pytest.raises(B.SvdqError):
         B.pack_weight_np("int4", R, None, None, 0.5)      # INT4 needs g_x = 1
+    with pytest.raises(B.SvdqError):
+        B.pack_weight_np("mxfp4", R, None, None, 2.0)     # MXFP4 has no tensor scale
 
 
 def test_selftest_rejects_limits_out_of_range():

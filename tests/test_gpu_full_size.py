@@ -98,8 +98,8 @@ def _sample_rows(M, seed):
     return np.array(sorted(rows))
 
 
-@pytest.mark.parametrize("name,fmt", [("mlp_up", "nvfp4"), ("mlp_up", "int4"), ("qkv", "nvfp4"),
-                                      ("mlp_down", "nvfp4"), ("mlp_down", "int4")])
+@pytest.mark.parametrize("name,fmt", [("mlp_up", "nvfp4"), ("mlp_up", "int4"), ("mlp_up", "mxfp4"), ("qkv", "nvfp4"),
+                                      ("mlp_down", "nvfp4"), ("mlp_down", "int4"), ("mlp_down", "mxfp4")])
 def test_full_size_layer_sampled_rows(name, fmt):
     cfg = I.NAMED[name]
     _run_and_check(cfg, fmt, _sample_rows(cfg.b, 7))

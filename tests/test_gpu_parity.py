@@ -61,7 +61,7 @@ def _check_prologue(fmt, X, lam, gx, L1_rk):
     return got, ref
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 @pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
                                       (96, 512, 128)])
 def test_prologue_parity(fmt, M, K, rank):
@@ -69,7 +69,7 @@ def test_prologue_parity(fmt, M, K, rank):
     _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 def test_prologue_without_smoothing_and_zero_rows(fmt):
     rng = np.random.default_rng(5)
     X = I.to_bf16(rng.standard_normal((200, 384)) * 3)
@@ -93,6 +93,24 @@ def test_prologue_rounding_ties_nvfp4():
     X = I.to_bf16(X)
     got, ref = _check_prologue("nvfp4", X, None, 1.0, None)
     assert got["codes"][0, 1] == 0 and got["codes"][0, 2] == 2 and got["codes"][0, 8] == 8
+
+
+def test_prologue_rounding_mxfp4_scales_ties_and_saturation():
+    """MXFP4: E8M0 byte from the group absmax exponent (including a zero group and a
+    subnormal-range group), E2M1 midpoints after the exact power-of-two scaling, and the
+    clamp of values in (6 X, 8 X) to 6."""
+    M, K = 128, 256
+    X = np.zeros((M, K), np.float32)
+    X[:, 0] = 7.0                                      # amax 7: X = 1, 7 -> 6
+    X[:, 1:9] = [0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.25]
+    X[:, 32] = 6.0 * 2.0 ** -20                        # second group: X = 2^-20
+    X[:, 33] = 2.5 * 2.0 ** -20
+    X[:, 64:96] = 0.0                                  # zero group: byte 0
+    X[:, 96] = 2.0 ** -127                             # tiny group: byte 0, code 0
+    X[:, 128] = -3.0 * 2.0 ** 30
+    X[:, 129] = 0.75 * 2.0 ** 30
+    X = I.to_bf16(X)
+    _check_prologue("mxfp4", X, None, 1.0, None)
 
 
 def test_prologue_rounding_ties_int4():
@@ -126,14 +144,14 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     return Yg, ref
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 @pytest.mark.parametrize("M,N,K,rank", [(300, 640, 640, 32), (256, 512, 512, 16), (128, 256, 256, 0),
                                         (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64)])
 def test_gemm_parity(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=11 + M + N + rank)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 @pytest.mark.parametrize("M,N,K,rank", [(2304, 3072, 512, 32), (2560, 2560, 256, 0), (2304, 3072, 256, 128),
                                         (1300, 3072, 768, 16)])
 def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
@@ -142,12 +160,12 @@ def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=5 + M + K + rank)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 def test_gemm_parity_no_bias(fmt):
     _gemm_case(fmt, 160, 512, 512, 32, seed=3, with_bias=False)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
 def test_gemm_lowrank_branch_is_added(fmt):
     """Y(r) - Y(r=0 on the same 4-bit operands) equals Z L2 (the branch really lands in Y)."""
     M, N, K, rank = 128, 256, 256, 32
@@ -165,7 +183,7 @@ def test_gemm_lowrank_branch_is_added(fmt):
 
 
 @pytest.mark.parametrize("fmt,rank", [("nvfp4", 32), ("nvfp4", 0), ("nvfp4", 128), ("int4", 32), ("int4", 0),
-                                      ("int4", 128)])
+                                      ("int4", 128), ("mxfp4", 32), ("mxfp4", 0), ("mxfp4", 128)])
 def test_layer_end_to_end_small(fmt, rank):
     """Prologue then GEMM on the device (Z never leaves the GPU) vs the reference layer."""
     M, K, N = 384, 768, 768
@@ -188,9 +206,10 @@ def test_layer_end_to_end_small(fmt, rank):
     ref_gz = O.gemm_forward(ref["q"], gx, packed["q"], packed["gscale"], got["Z"], packed["L2_bf16"], layer.bias)
     assert rel_fro(Yg, ref_gz["Y"]) <= Y_TOL
     assert rel_fro(Yg, ref["Y"]) <= 2e-3
-    # and the layer approximates the unquantized X W + b
+    # and the layer approximates the unquantized X W + b (MXFP4's power-of-two scales clamp
+    # values in (6 X, 8 X), so its plain W4A4 error, at rank 0, is the largest)
     exact = layer.X.astype(np.float64) @ layer.W + layer.bias.astype(np.float64)
-    assert rel_fro(Yg, exact) < 0.15
+    assert rel_fro(Yg, exact) < (0.25 if fmt == "mxfp4" else 0.15)
 
 
 def _finite_bf16_values(lo=1e-30, hi=1e30):
