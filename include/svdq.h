@@ -84,8 +84,8 @@ typedef enum {
    * as its E8M0 byte: X = 2^(floor(log2 a) - 2), clamped to [2^-127, 2^127], the MX
    * shared scale of the OCP Microscaling format for E2M1 (largest value 6 = 1.5 * 2^2);
    * q = e2m1_satfinite(x / X).  No tensor scale: act_gscale and w_gscale are 1.
-   * ("SVDQuant（实验性功能）": the Nunchaku export uses MXFP4 E2M1 W4A4, group size 32,
-   * symmetric.) */
+   * ("SVDQuant（实验性功能）": its Nunchaku export needs E2M1 weights and activations in
+   * 32-element groups, quantized symmetrically.) */
   SVDQ_FMT_MXFP4_G32 = 3
 } svdq_format;
 

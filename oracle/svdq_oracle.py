@@ -45,8 +45,9 @@ Readings where the pages are silent (each one is listed in the design doc):
    to bf16); it feeds both the quantizer and the down projection.  L1, L2 and
    Z are bf16.
 8. Sigma goes into L1 (eq.(10) of *SVDQuant 阅读笔记*).
-9. MXFP4 (*AutoRound SVDQuant*, the Nunchaku export: "MXFP4 E2M1 W4A4, group size 32,
-   symmetric"): the MX shared scale of the OCP Microscaling format,
+9. MXFP4 (*AutoRound SVDQuant*: its Nunchaku export needs E2M1 weights and activations in
+   32-element groups, quantized symmetrically): the MX shared scale of the OCP Microscaling
+   format,
    ``X = 2 ** clip(floor(log2(amax)) - 2, -127, 127)`` (2 = exponent of the largest
    E2M1 value 6), stored as its E8M0 byte ``log2(X) + 127``; ``q = e2m1_rn_satfinite(x / X)``
    (the divide is exact).  ``amax == 0`` gives byte 0.  No tensor scale (g = 1).
