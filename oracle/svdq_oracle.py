@@ -25,7 +25,7 @@ Sources (cited by page title and section / equation):
   cited as *msModelSlim SVDQuant*), "SVD 分解过程": factor shapes
   ``l1 = V^T`` [rank, in] and ``l2 = U S`` [out, rank]; "前向等价关系".
 
-Readings where the pages are silent (each one is listed in the design doc):
+Readings where the pages are silent:
 
 1. ``round`` in eq.(1) is round-half-to-even (``np.rint``).
 2. INT4 scale: ``s = fp16_rn(fp32(a / 7))`` (saturating at 65504), and the
