@@ -54,6 +54,10 @@ def parse_args():
                     help="svd: smoothing + SVD split of the synthetic W (default); random: seeded random "
                          "R, L1, L2 of the same shapes and scale, no decomposition (for short profiler runs; "
                          "the kernels' time and traffic do not depend on the weight values)")
+    ap.add_argument("--residual-iters", type=int, default=1,
+                    help="outer residual iterations of the offline split (1: plain SVD split)")
+    ap.add_argument("--residual-early-stop", action="store_true",
+                    help="keep the best residual-iteration candidate and stop once the target gets worse")
     return ap.parse_args()
 
 
@@ -77,12 +81,19 @@ def workload(args):
     return cfg
 
 
-def prepare_layer(cfg, fmt, device, weights="svd"):
+def prepare_layer(cfg, fmt, device, weights="svd", residual_iters=1, early_stop=False):
     from bit_w4a4_quantized_group_b200 import inputs as I
     from bit_w4a4_quantized_group_b200 import prepare as P
     layer = I.make_layer(cfg)
     if weights == "svd":
-        prep = P.prepare(fmt, layer.X, layer.W, cfg.rank, device=device)
+        if device.startswith("cuda"):
+            torch.cuda.synchronize()
+        t0 = time.perf_counter()
+        prep = P.prepare(fmt, layer.X, layer.W, cfg.rank, device=device,
+                         residual_iters=residual_iters, early_stop=early_stop)
+        if device.startswith("cuda"):
+            torch.cuda.synchronize()
+        prep["offline_s"] = time.perf_counter() - t0
     else:
         rng = np.random.default_rng(cfg.seed + 1000)
         K, N, r = cfg.m, cfg.n, cfg.rank
@@ -357,7 +368,8 @@ def main():
 
     cfg = workload(args)
     fmt = args.format
-    layer, prep, packed = prepare_layer(cfg, fmt, str(device), args.weights)
+    layer, prep, packed = prepare_layer(cfg, fmt, str(device), args.weights, args.residual_iters,
+                                        args.residual_early_stop)
     M, K, N, r = cfg.b, cfg.m, cfg.n, cfg.rank
     lin = W4A4LowRankLinear(fmt, N, K, packed, prep["lam"], prep["act_gscale"], layer.bias, device=device)
     from bit_w4a4_quantized_group_b200.inputs import bf16_bits
@@ -531,6 +543,13 @@ def main():
         "gpu_launches": launches,
         "clocks": clk,
     }
+    if "offline_s" in prep:
+        res = prep.get("residual") or {}
+        out["offline_split"] = {
+            "seconds": prep["offline_s"], "where": str(device), "residual_iters": args.residual_iters,
+            "early_stop": args.residual_early_stop, "chosen": res.get("chosen", 0),
+            "output_errors": res.get("errors"),
+            "note": "smoothing + fp64 SVD split (+ residual iterations), untimed setup, not part of value"}
     if e2e:
         out["e2e"] = {"value": whole_job_tflops(world, flops, t_e2e), "unit": UNIT, "h2d_bytes_per_step": e2e["h2d"],
                       "d2h_bytes_per_step": e2e["d2h"]}

@@ -67,6 +67,7 @@ __all__ = [
     "dequantize", "quantize", "prologue", "pack_weight", "w4a4_main", "gemm_forward",
     "layer_forward", "prepare_layer", "rho_mac", "rho_bytes", "prop41_bound",
     "brute_force_w4a4", "INT4_QMAX", "NVFP4_QMAX", "E4M3_MAX", "quantize_mxfp4_g32", "MXFP4_EMAX",
+    "residual_iteration",
 ]
 
 INT4_QMAX = 7          # eq.(1): symmetric codes -7..7
@@ -239,6 +240,53 @@ def svd_split(W_tilde: np.ndarray, rank: int):
         "R64": R64, "R": R64.astype(np.float32), "sigma": S,
         "R_exact": W_tilde - L1 @ L2,
     }
+
+
+def residual_iteration(fmt: str, W_tilde: np.ndarray, rank: int, iters: int,
+                       early_stop: bool = False, X_hat: Optional[np.ndarray] = None):
+    """AutoRound "SVDQuant（实验性功能）", "Residual iteration": alternate a low-rank fit
+    with the deployment RTN quantize-dequantize of the residual (reading 17).
+
+    Iteration 0 is the plain split of eq.(10): L1 L2 = SVD_r(W_tilde), R = W_tilde - L1 L2
+    with bf16 factors.  Each further outer iteration fits the branch to W_tilde - Q(R_prev),
+    forms the new residual R = W_tilde - L1 L2 and quantize-dequantizes it as it is deployed
+    (per output channel along the input dimension, with the tensor scale of reading 4 for
+    NVFP4).  The target error is the weight reconstruction error ||L1 L2 + Q(R) - W_tilde||_F,
+    or, with calibration activations X_hat (smoothing on), the calibration output error
+    ||X_hat (L1 L2 + Q(R) - W_tilde)||_F.  With early_stop the best candidate so far is kept
+    and the loop ends at the first candidate whose error is worse; without it all iterations
+    run and the last candidate is returned.
+    """
+    W_tilde = np.asarray(W_tilde, dtype=np.float64)
+    Xh = None if X_hat is None else np.asarray(X_hat, dtype=np.float64)
+
+    def qdq(R32):
+        gw = pow2_global_scale(np.max(np.abs(R32)) if R32.size else 0.0) if fmt == "nvfp4" else 1.0
+        return dequantize(fmt, quantize(fmt, np.ascontiguousarray(R32.T), gw)).T
+
+    def target(L1b, L2b, QR):
+        E = L1b @ L2b + QR - W_tilde
+        return float(np.linalg.norm(E if Xh is None else Xh @ E))
+
+    sp = svd_split(W_tilde, rank)
+    cand = (sp["L1_bf16"], sp["L2_bf16"], sp["R"])
+    QR = qdq(cand[2])
+    errs = [target(cand[0], cand[1], QR)]
+    best, best_err, best_it = cand, errs[0], 0
+    for it in range(1, max(int(iters), 1)):
+        fit = svd_split(W_tilde - QR, rank)
+        L1b, L2b = fit["L1_bf16"], fit["L2_bf16"]
+        cand = (L1b, L2b, (W_tilde - L1b @ L2b).astype(np.float32))
+        QR = qdq(cand[2])
+        errs.append(target(L1b, L2b, QR))
+        if early_stop:
+            if errs[-1] < best_err:
+                best, best_err, best_it = cand, errs[-1], it
+            else:
+                break
+        else:
+            best, best_err, best_it = cand, errs[-1], it
+    return {"L1_bf16": best[0], "L2_bf16": best[1], "R": best[2], "chosen": best_it, "errors": errs}
 
 
 def lora_concat(L1: np.ndarray, L2: np.ndarray, lam: Optional[np.ndarray],
@@ -426,16 +474,25 @@ def layer_forward(fmt: str, X, lam, act_gscale, packed, bias=None):
 
 
 def prepare_layer(fmt: str, X_calib: np.ndarray, W: np.ndarray, rank: int,
-                  alpha: float = 0.5, smooth: bool = True, lora=None):
+                  alpha: float = 0.5, smooth: bool = True, lora=None,
+                  residual_iters: int = 1, early_stop: bool = False):
     """Offline build of one layer: lambda (eq.(4)), W_tilde (eq.(3)), SVD split (eq.(10)).
 
-    Returns the ABI-orientation arrays: R_nk [N, K] fp32, L1_rk [r, K] and
-    L2_nr [N, r] (fp64 values of the bf16 factors), lambda [K] fp32 and the
-    activation tensor scale g_x (reading 4, from the calibration X_hat).
+    With residual_iters > 1 the split is refined by ``residual_iteration``, whose
+    target is the calibration output error when smoothing is on and the weight
+    reconstruction error when it is off.  Returns the ABI-orientation arrays:
+    R_nk [N, K] fp32, L1_rk [r, K] and L2_nr [N, r] (fp64 values of the bf16
+    factors), lambda [K] fp32 and the activation tensor scale g_x (reading 4,
+    from the calibration X_hat).
     """
     lam = smoothing_factors(X_calib, W, alpha) if smooth else None
     Wt = smooth_weight(W, lam)
-    sp = svd_split(Wt, rank)
+    if residual_iters > 1:
+        ri = residual_iteration(fmt, Wt, rank, residual_iters, early_stop,
+                                smooth_activations(X_calib, lam) if smooth else None)
+        sp = {"L1_bf16": ri["L1_bf16"], "L2_bf16": ri["L2_bf16"], "R": ri["R"], "residual": ri}
+    else:
+        sp = svd_split(Wt, rank)
     L1, L2 = sp["L1_bf16"], sp["L2_bf16"]
     if lora is not None:
         L1, L2 = lora_concat(L1, L2, lam, lora[0], lora[1])
