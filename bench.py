@@ -431,9 +431,10 @@ def main():
     torch.cuda.synchronize()
     t_gemm0 = sum(a.elapsed_time(b) for a, b in gemm0) / len(gemm0) * 1e-3
     # Fusion: the layer without the branch (prologue and GEMM at rank 0), and the same layer
-    # with an unfused branch as separate passes (msModelSlim's "residual_out +
-    # F.linear(F.linear(x, l1), l2)" form): X / lambda -> bf16, Z = X_hat L1^T, Y += Z L2^T,
-    # the low-rank products on cuBLAS in bf16.  Reported beside the headline, not part of it.
+    # with an unfused branch as separate passes (msModelSlim's two-path forward: the residual
+    # linear's output plus two chained low-rank linears): X / lambda -> bf16, Z = X_hat L1^T,
+    # Y += Z L2^T, the low-rank products on cuBLAS in bf16.  Reported beside the headline,
+    # not part of it.
     fusion = None
     if r > 0:
         lam_d = lin.lam if lin.lam is not None else torch.ones(K, device=device)
