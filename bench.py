@@ -84,6 +84,7 @@ def workload(args):
 def prepare_layer(cfg, fmt, device, weights="svd", residual_iters=1, early_stop=False):
     from bit_w4a4_quantized_group_b200 import inputs as I
     from bit_w4a4_quantized_group_b200 import prepare as P
+    import torch
     layer = I.make_layer(cfg)
     if weights == "svd":
         if device.startswith("cuda"):
