@@ -51,6 +51,12 @@ Readings where the pages are silent:
    ``X = 2 ** clip(floor(log2(amax)) - 2, -127, 127)`` (2 = exponent of the largest
    E2M1 value 6), stored as its E8M0 byte ``log2(X) + 127``; ``q = e2m1_rn_satfinite(x / X)``
    (the divide is exact).  ``amax == 0`` gives byte 0.  No tensor scale (g = 1).
+10. W8A8 (*SVDQuant 阅读笔记* §8, the appendix-D 8-bit setting: rank 16, activations
+    quantized per token and dynamically, weights per output channel): eq.(1) with the
+    8-bit symmetric range, one group per row spanning all of K:
+    ``s = fp32(amax / 127)``, ``q = clamp(rint(fp32(x / s)), -127, 127)``; ``s == 0``
+    gives ``q = 0``.  The scale is kept in fp32 (the pages give no precision for it).
+    No tensor scale (g = 1).
 """
 from __future__ import annotations
 
@@ -67,13 +73,14 @@ __all__ = [
     "dequantize", "quantize", "prologue", "pack_weight", "w4a4_main", "gemm_forward",
     "layer_forward", "prepare_layer", "rho_mac", "rho_bytes", "prop41_bound",
     "brute_force_w4a4", "INT4_QMAX", "NVFP4_QMAX", "E4M3_MAX", "quantize_mxfp4_g32", "MXFP4_EMAX",
-    "residual_iteration",
+    "residual_iteration", "quantize_int8_rowwise", "INT8_QMAX",
 ]
 
 INT4_QMAX = 7          # eq.(1): symmetric codes -7..7
 NVFP4_QMAX = 6.0       # largest E2M1 magnitude
 E4M3_MAX = 448.0       # largest finite E4M3 magnitude
 MXFP4_EMAX = 2         # exponent of the largest E2M1 magnitude: 6 = 1.5 * 2^2
+INT8_QMAX = 127        # eq.(1) with 8 bits: symmetric codes -127..127
 
 
 # ---------------------------------------------------------------------------
@@ -380,7 +387,29 @@ def quantize_mxfp4_g32(x: np.ndarray):
             "scale": X, "scale_bits": (e + 127).astype(np.uint8), "gscale": 1.0}
 
 
+def quantize_int8_rowwise(x: np.ndarray):
+    """eq.(1) with 8-bit codes and one group per row (reading 10): per-token activations,
+    per-output-channel weights.
+
+    s = fp32(max|x_row| / 127) kept in fp32;  q = clamp(rint(fp32(x / s)), -127, 127).
+    Returns codes as uint8 two's-complement bytes [rows, K], the integer values, the
+    fp32 scale per row (as a [rows, 1] array) and its bits.
+    """
+    x = np.asarray(x, dtype=np.float32)
+    a = np.max(np.abs(x), axis=1, keepdims=True) if x.shape[1] else np.zeros((x.shape[0], 1), np.float32)
+    s = (a / np.float32(INT8_QMAX)).astype(np.float32)
+    safe = np.where(s > 0, s, np.float32(1.0))
+    v = (x / safe).astype(np.float32)
+    q = np.clip(np.rint(v), -INT8_QMAX, INT8_QMAX)
+    q = np.where(s > 0, q, 0.0)
+    codes = (q.astype(np.int64) & 0xFF).astype(np.uint8)
+    return {"codes": codes, "q": q.astype(np.float64), "scale": s,
+            "scale_bits": s.view(np.uint32), "gscale": 1.0}
+
+
 def quantize(fmt: str, x: np.ndarray, gscale: float = 1.0):
+    if fmt == "w8a8":
+        return quantize_int8_rowwise(x)
     if fmt == "int4":
         return quantize_int4_g64(x)
     if fmt == "nvfp4":
@@ -390,15 +419,18 @@ def quantize(fmt: str, x: np.ndarray, gscale: float = 1.0):
     raise ValueError(fmt)
 
 
-def group_size(fmt: str) -> int:
+def group_size(fmt: str, K: Optional[int] = None) -> int:
+    """Elements per scale along K; W8A8 has one scale per row (the whole of K)."""
+    if fmt == "w8a8":
+        return K
     return {"int4": 64, "nvfp4": 16, "mxfp4": 32}[fmt]
 
 
 def dequantize(fmt: str, qd) -> np.ndarray:
     """Q(Z) = g * s * q (fp64, exact)."""
-    gsz = group_size(fmt)
     q = qd["q"]
     rows, K = q.shape
+    gsz = group_size(fmt, K)
     s = np.repeat(qd["scale"].astype(np.float64), gsz, axis=1)
     return qd["gscale"] * s * q
 
@@ -437,7 +469,7 @@ def pack_weight(fmt: str, R_nk: np.ndarray, L1_rk: np.ndarray, L2_nr: np.ndarray
     if fmt == "nvfp4":
         gw = pow2_global_scale(np.max(np.abs(R_nk)) if R_nk.size else 0.0)
     else:
-        gw = 1.0      # INT4 and MXFP4 have no tensor scale
+        gw = 1.0      # INT4, MXFP4 and W8A8 have no tensor scale
     qd = quantize(fmt, R_nk, gw)
     L1b = bf16_rn(L1_rk)
     L2b = bf16_rn(L2_nr)
@@ -531,8 +563,8 @@ def prop41_bound(X, W, QX, QW):
 
 def brute_force_w4a4(fmt: str, qa, qw) -> np.ndarray:
     """Triple loop over (i, j, k) with per-element dequantization (tiny shapes only)."""
-    gsz = group_size(fmt)
     M, K = qa["q"].shape
+    gsz = group_size(fmt, K)
     N = qw["q"].shape[0]
     out = np.zeros((M, N))
     for i in range(M):

@@ -317,3 +317,87 @@ def test_mxfp4_dequant_error_bound():
     a = np.repeat(np.abs(x.reshape(16, 32, 32)).max(-1), 32, axis=1)
     # half the largest E2M1 gap (1) times X, plus the clamp of values in (6 X, 8 X)
     assert np.all(np.abs(x - deq) <= X * 1.0 + np.maximum(a - 6 * X, 0) + 1e-12)
+
+
+# ------------------------------------------------------- W8A8 per row (reading 10)
+
+def test_int8_rowwise_worked_example_eq1_with_8_bits():
+    """eq.(1) with the symmetric 8-bit range: max 127 gives step 1; max 1 gives step 1/127."""
+    x = np.zeros((2, 128), np.float32)
+    x[0, 0] = 127.0
+    x[0, 1:6] = [0.4, -0.6, 2.5, 3.5, -126.5]        # 0.4 -> 0, ties to even: 2, 4, -126
+    x[1, 0] = -1.0
+    x[1, 1] = 0.5
+    q = O.quantize_int8_rowwise(x)
+    assert q["scale"][0, 0] == 1.0
+    assert list(q["q"][0, :6]) == [127, 0, -1, 2, 4, -126]
+    assert q["scale"][1, 0] == np.float32(1.0) / np.float32(127.0)
+    assert q["q"][1, 0] == -127
+    assert q["codes"][1, 0] == 0x81 and q["codes"][0, 0] == 0x7F and q["codes"][0, 2] == 0xFF
+    # 0.5 / fp32(1/127) = 63.5 up to the fp32 rounding of the scale and of the quotient
+    assert q["q"][1, 1] in (63.0, 64.0)
+    assert q["q"][1, 1] == np.rint(np.float32(0.5) / q["scale"][1, 0])
+
+
+def test_int8_rowwise_codes_are_nearest_and_bounded():
+    """Against exact rational arithmetic: q is the nearest integer to x/s except within
+    the fp32 quotient's rounding of a midpoint; |x - s q| <= s/2 up to that rounding."""
+    from fractions import Fraction
+    rng = np.random.default_rng(31)
+    x = O.bf16_rn(rng.standard_normal((24, 256)) * np.exp2(rng.integers(-30, 30, (24, 1))))
+    x[3] = 0.0
+    q = O.quantize_int8_rowwise(x)
+    assert np.all(q["q"][3] == 0) and q["scale"][3, 0] == 0
+    for i in range(24):
+        if i == 3:
+            continue
+        a = Fraction(float(np.abs(x[i]).max()))
+        s = Fraction(float(q["scale"][i, 0]))
+        assert abs(s - a / 127) <= s * Fraction(1, 2 ** 24)          # s = fp32 of amax / 127
+        for k in range(0, 256, 7):
+            t = Fraction(float(x[i, k])) / s
+            qi = int(q["q"][i, k])
+            assert -127 <= qi <= 127
+            assert abs(t - qi) <= Fraction(1, 2) + abs(t) * Fraction(1, 2 ** 23)
+        # the max element maps to +-127
+        j = int(np.argmax(np.abs(x[i])))
+        assert abs(int(q["q"][i, j])) == 127
+
+
+def test_int8_rowwise_matches_torch_fp32_semantics():
+    """rint(fp32(x / s)) checked against torch's IEEE fp32 divide and round-half-even."""
+    import torch
+    rng = np.random.default_rng(32)
+    x = O.bf16_rn(rng.standard_normal((16, 512)) * np.exp2(rng.integers(-10, 10, (16, 1))))
+    x[5, :4] = [127.0, 63.5, -0.5, 1.5]           # exact midpoints with s = 1
+    x[5, 4:] = 0.0
+    q = O.quantize_int8_rowwise(x)
+    xt = torch.from_numpy(x)
+    st = (xt.abs().amax(1, keepdim=True) / 127.0)
+    assert np.array_equal(st.numpy(), q["scale"])
+    qt = torch.clamp(torch.round(xt / st), -127, 127)
+    assert np.array_equal(qt.numpy().astype(np.float64), q["q"])
+    assert list(q["q"][5, :4]) == [127, 64, -0.0, 2]
+
+
+def test_int8_rowwise_sign_symmetry_and_power_of_two_equivariance():
+    rng = np.random.default_rng(33)
+    x = O.bf16_rn(rng.standard_normal((8, 384)))
+    q0 = O.quantize_int8_rowwise(x)
+    qn = O.quantize_int8_rowwise(-x)
+    assert np.array_equal(qn["q"], -q0["q"]) and np.array_equal(qn["scale"], q0["scale"])
+    for k in (-40, -3, 5, 60):
+        qk = O.quantize_int8_rowwise((x * np.float32(2.0 ** k)).astype(np.float32))
+        assert np.array_equal(qk["q"], q0["q"])
+        assert np.array_equal(qk["scale"], (q0["scale"] * np.float32(2.0 ** k)).astype(np.float32))
+
+
+def test_int8_rowwise_dequant_is_per_row_scale_times_code():
+    rng = np.random.default_rng(34)
+    x = O.bf16_rn(rng.standard_normal((4, 256)))
+    q = O.quantize_int8_rowwise(x)
+    deq = O.dequantize("w8a8", q)
+    for i in range(4):
+        for k in (0, 17, 255):
+            assert deq[i, k] == float(q["scale"][i, 0]) * int(np.int8(q["codes"][i, k]))
+    assert np.all(np.abs(x - deq) <= q["scale"].astype(np.float64) * (0.5 + 2.0 ** -16))
