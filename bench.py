@@ -46,7 +46,9 @@ def parse_args():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="svdq", choices=["svdq", "reference"])
     ap.add_argument("--workload", default="mlp_up")
-    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "int4", "mxfp4"])
+    ap.add_argument("--format", default="nvfp4", choices=["nvfp4", "int4", "mxfp4", "w8a8"],
+                    help="w8a8 is the 8-bit setting (per-token activations, per-channel weights); "
+                         "its rank defaults to 16")
     ap.add_argument("--rank", type=int, default=None)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -75,6 +77,8 @@ def peaks():
 def workload(args):
     from bit_w4a4_quantized_group_b200 import inputs as I
     cfg = I.NAMED[args.workload]
+    if args.rank is None and args.format == "w8a8":
+        args.rank = 16                       # the 8-bit setting's rank
     if args.rank is not None and args.rank != cfg.rank:
         import dataclasses
         cfg = dataclasses.replace(cfg, rank=args.rank)
@@ -515,13 +519,19 @@ def main():
     else:
         peak = bf16_burst * 2.0              # dense INT8 = 2 x dense bf16 (nominal ratio 4.5 : 2.25)
         peak_note = f"dense INT8 = 2 x {peak_src} bf16 burst"
-        src = os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc", "gemm_int4.cu")
+        src = os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc",
+                           "gemm_w8a8.cu" if fmt == "w8a8" else "gemm_int4.cu")
     alg_flops = flops + 2.0 * M * N * r
     achieved = alg_flops / t_gemm / 1e12
     traffic = recorded_traffic(src, f"{cfg.name}_{fmt}_r{r}")
-    g = {"nvfp4": 16, "mxfp4": 32, "int4": 64}[fmt]
-    sf = 2 if fmt == "int4" else 1
-    pro_bytes = 2 * M * K + M * K / 2 + M * K / g * sf + 2 * M * r + 2 * r * K + (4 * K)
+    if fmt == "w8a8":
+        # algorithmic bytes: X once (the kernel's second pass over X is served mostly from
+        # L2), one byte per code, one fp32 scale per row
+        pro_bytes = 2 * M * K + M * K + 4 * M + 2 * M * r + 2 * r * K + (4 * K)
+    else:
+        g = {"nvfp4": 16, "mxfp4": 32, "int4": 64}[fmt]
+        sf = 2 if fmt == "int4" else 1
+        pro_bytes = 2 * M * K + M * K / 2 + M * K / g * sf + 2 * M * r + 2 * r * K + (4 * K)
     out = {
         "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",

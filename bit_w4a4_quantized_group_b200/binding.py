@@ -18,7 +18,9 @@ SVDQ_OK, SVDQ_ERR_INVALID_ARG, SVDQ_ERR_UNSUPPORTED, SVDQ_ERR_CUDA, SVDQ_ERR_TIM
 SVDQ_FMT_NVFP4_G16 = 1
 SVDQ_FMT_INT4_G64 = 2
 SVDQ_FMT_MXFP4_G32 = 3
-FORMATS = {"nvfp4": SVDQ_FMT_NVFP4_G16, "int4": SVDQ_FMT_INT4_G64, "mxfp4": SVDQ_FMT_MXFP4_G32}
+SVDQ_FMT_W8A8 = 4
+FORMATS = {"nvfp4": SVDQ_FMT_NVFP4_G16, "int4": SVDQ_FMT_INT4_G64, "mxfp4": SVDQ_FMT_MXFP4_G32,
+           "w8a8": SVDQ_FMT_W8A8}
 
 EXPORTED = (
     "svdq_buffer_sizes", "svdq_pack_weight", "svdq_quantize_act_lowrank_down",

@@ -91,19 +91,6 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
          (static_cast<uint32_t>(m >> 4) << 24);
 }
 
-// Tile schedule: cluster c takes the contiguous run [begin, begin + count) of the N-fastest
-// tile numbering, so consecutive tiles of a cluster share the M block.
-struct TileSeq {
-  int begin, count, tiles_n;
-  __device__ TileSeq(int num_tiles, int tiles_n_, int cluster, int nclusters) : tiles_n(tiles_n_) {
-    const int base = num_tiles / nclusters, extra = num_tiles % nclusters;
-    begin = cluster * base + min(cluster, extra);
-    count = base + (cluster < extra ? 1 : 0);
-  }
-  __device__ int mb(int j) const { return (begin + j) / tiles_n; }
-  __device__ int nb(int j) const { return (begin + j) % tiles_n; }
-};
-
 struct SharedTail {
   uint64_t full[kStages];
   uint64_t empty[kStages];

@@ -4,7 +4,8 @@
 // steps 5 and 9: the residual R is quantized with the deployment format and
 // saved together with the low-rank factors.  Formats follow §2.2 and §8 of
 // the same page: INT4 groups of 64 with a 16-bit scale (eq.(1), s = max|Z|/7),
-// NVFP4 groups of 16 with an FP8 (E4M3) scale.  The rounding rules are the
+// NVFP4 groups of 16 with an FP8 (E4M3) scale; the 8-bit setting of §8 (appendix D)
+// quantizes each output channel of the weight with one scale (W8A8).  The rounding rules are the
 // ones stated in svdq.h; every conversion below is written from the format
 // definition (IEEE binary16, bfloat16, OCP E4M3 "fn", E2M1).
 #include <algorithm>
@@ -149,11 +150,27 @@ extern "C" svdq_status svdq_pack_weight(svdq_format fmt, int64_t N, int64_t K, i
   if (fmt != SVDQ_FMT_NVFP4_G16 && act_gscale != 1.0f) return SVDQ_ERR_INVALID_ARG;
 
   uint8_t* codes = static_cast<uint8_t*>(w_codes);
-  std::memset(codes, 0, static_cast<size_t>(N) * static_cast<size_t>(K / 2));
+  std::memset(codes, 0, code_bytes(fmt, N, K));
   const int64_t Np = (N + 127) / 128 * 128;
 
   float gw = 1.0f;
-  if (fmt == SVDQ_FMT_NVFP4_G16) {
+  if (fmt == SVDQ_FMT_W8A8) {
+    // one scale per output channel: s = fp32(a / 127), q = clamp(rint(fp32(x / s)), -127, 127)
+    float* sf = static_cast<float*>(w_scales);
+    std::memset(sf, 0, static_cast<size_t>(Np) * sizeof(float));
+    for (int64_t n = 0; n < N; ++n) {
+      const float* row = R + n * K;
+      float a = 0.0f;
+      for (int64_t k = 0; k < K; ++k) a = std::fmax(a, std::fabs(row[k]));
+      const float s = a / 127.0f;
+      sf[n] = s;
+      for (int64_t k = 0; k < K; ++k) {
+        int q = 0;
+        if (s > 0.0f) q = static_cast<int>(std::fmax(-127.0f, std::fmin(127.0f, std::nearbyint(row[k] / s))));
+        codes[n * K + k] = static_cast<uint8_t>(q & 0xFF);
+      }
+    }
+  } else if (fmt == SVDQ_FMT_NVFP4_G16) {
     float amax = 0.0f;
     for (int64_t i = 0; i < N * K; ++i) amax = std::fmax(amax, std::fabs(R[i]));
     gw = pow2_gscale(amax);

@@ -16,6 +16,13 @@
 // shared memory and written back as 16-byte row segments.  Z partials of the
 // warps that share a row strip are summed in a fixed order (deterministic).
 //
+// W8A8 (the 8-bit setting: one scale per token row over all of K) needs each row's
+// maximum before any code can be formed, so the kernel makes two passes over its rows:
+// the first forms X_hat, the Z products and the row maxima; the compute warps then
+// combine their maxima and write the fp32 row scales; the second pass re-reads X (the
+// CTAs' rows were just read, so the L2 serves most of it), re-forms X_hat and writes
+// one-byte codes with an IEEE-exact divide by the row scale.
+//
 // Divisions are IEEE-exact without the divide instruction sequence:
 //  * X / lambda uses Markstein's correction (P. Markstein, "Computation of
 //    elementary functions on the IBM RISC System/6000 processor", IBM J. Res.
@@ -107,6 +114,10 @@ __device__ __forceinline__ float div_code(float a, float b, float y) {
   return fmaf(-fmaf(b, q0, -a), y, q0);
 }
 
+// Bytes of code staging per compute warp: 16 rows x 64 columns of 4-bit or 8-bit codes.
+__host__ __device__ constexpr int code_stage_bytes(int fmt) { return fmt == kFmtW8a8 ? 1024 : 512; }
+__host__ __device__ constexpr int passes(int fmt) { return fmt == kFmtW8a8 ? 2 : 1; }
+
 template <int FMT, int RANK>
 __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_l1,
@@ -122,8 +133,11 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   const int S = p.stages;
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S * L.stage_bytes);
   uint64_t* empty = full + S;
-  uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // NW warps x 512 B code staging
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(cstage + NW * 512);
+  constexpr int CSTB = code_stage_bytes(FMT);
+  constexpr int NPASS = passes(FMT);
+  uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // NW warps x CSTB code staging
+  float* rmax_s = reinterpret_cast<float*>(cstage + NW * CSTB);     // W8A8: [BOXES][2 strips][16 rows]
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(rmax_s + BOXES * 32);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -160,10 +174,13 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       }
     };
     load_lambda(kt0 % nkt);
-    for (int ki = 0; ki < nkt; ++ki) {
-      const int s = ki % S;
-      const uint32_t ph = (ki / S) & 1;
+    const int nit = NPASS * nkt;
+    for (int it = 0; it < nit; ++it) {
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
       if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
+      const int ki = it % nkt;
+      const bool with_l1 = RANK > 0 && it < nkt;      // L1 is only needed by the first pass
       const int kt = (kt0 + ki) % nkt;
       const int col0 = kt * BK;
       const int nbox = min(BK, p.K - col0) / 64;
@@ -173,16 +190,16 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       if (lane == 0) {
         // kProBoxes boxes per load; boxes past K are zero-filled and counted like the others
         const int nload = (nbox + kProBoxes - 1) / kProBoxes;
-        ptx::mbar_expect_tx(&full[s], nload * kProBoxes * (kXBoxBytes + 128u * RANK));
+        ptx::mbar_expect_tx(&full[s], nload * kProBoxes * (kXBoxBytes + (with_l1 ? 128u * RANK : 0u)));
         for (int b = 0; b < nload * kProBoxes; b += kProBoxes) {
           ptx::tma_load_3d(st + L.x_off + b * kXBoxBytes, &tmap_x, &full[s], 0, m0, col0 / 64 + b);
-          if (RANK > 0) ptx::tma_load_3d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], 0, 0, col0 / 64 + b);
+          if (with_l1) ptx::tma_load_3d(st + L.l1_off + b * 128 * RANK, &tmap_l1, &full[s], 0, 0, col0 / 64 + b);
         }
       }
       float cur[BK / 32];
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) cur[i] = lv[i];
-      if (ki + 1 < nkt) load_lambda((kt0 + ki + 1) % nkt);
+      if (it + 1 < nit) load_lambda((kt0 + (it + 1) % nkt) % nkt);
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) {
         lam_s[i * 32 + lane] = cur[i];
@@ -200,16 +217,23 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     float acc[NT > 0 ? NT : 1][4];
 #pragma unroll
     for (int i = 0; i < (NT > 0 ? NT : 1); ++i) acc[i][0] = acc[i][1] = acc[i][2] = acc[i][3] = 0.f;
-    uint8_t* cst = cstage + warp * 512;
+    uint8_t* cst = cstage + warp * CSTB;
     const int K2 = p.K / 2;
     const float gs = p.gscale;
     const float inv_gs = 1.0f / gs;     // exact: gs is a power of two
     constexpr float kRcp6 = 1.0f / 6.0f, kRcp7 = 1.0f / 7.0f;
     bool ok = true;
+    // W8A8: running max |x_hat| of rows row_a / row_b over this warp's boxes (first pass), then
+    // the row scales as divisors for the second pass: x_hat / s is formed as (x_hat f) / (s f)
+    // with f = 2^64 for scales below 2^-64 (exact), so that RN(1 / (s f)) stays finite
+    float rmax_a = 0.f, rmax_b = 0.f;
+    float w8_fa = 1.f, w8_fb = 1.f, w8_ba = 0.f, w8_bb = 0.f, w8_nya = 0.f, w8_nyb = 0.f;  // b = 0: zero codes
 
+    for (int pass = 0; pass < NPASS; ++pass) {
     for (int ki = 0; ki < nkt && ok; ++ki) {
-      const int s = ki % S;
-      const uint32_t ph = (ki / S) & 1;
+      const int it = pass * nkt + ki;
+      const int s = it % S;
+      const uint32_t ph = (it / S) & 1;
       if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
       const int kt = (kt0 + ki) % nkt;
       const int col0 = kt * BK + phase * 64;
@@ -246,9 +270,9 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           nx[j][1] = neg_bf16x2(ah[2]);
           nx[j][2] = neg_bf16x2(ah[1]);
           nx[j][3] = neg_bf16x2(ah[3]);
-          // low-rank down projection on the tensor cores
+          // low-rank down projection on the tensor cores (first pass only)
 #pragma unroll
-          for (int nt2 = 0; nt2 < NT / 2; ++nt2) {
+          for (int nt2 = 0; nt2 < (pass == 0 ? NT / 2 : 0); ++nt2) {
             uint32_t b[4];
             const int n = nt2 * 16 + (lane & 7) + ((lane >> 4) & 1) * 8;
             const int ch = 2 * j + ((lane >> 3) & 1);
@@ -387,6 +411,38 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
             sc[static_cast<size_t>(grp) * p.Mpad + row_a] = ha;
             sc[static_cast<size_t>(grp) * p.Mpad + row_b] = hb;
           }
+        } else if (FMT == kFmtW8a8) {
+          if (pass == 0) {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              rmax_a = fmaxf(rmax_a, fmaxf(fmaxf(fabsf(nx[j][0].x), fabsf(nx[j][0].y)), fmaxf(fabsf(nx[j][1].x), fabsf(nx[j][1].y))));
+              rmax_b = fmaxf(rmax_b, fmaxf(fmaxf(fabsf(nx[j][2].x), fabsf(nx[j][2].y)), fmaxf(fabsf(nx[j][3].x), fabsf(nx[j][3].y))));
+            }
+          } else {
+            // q = clamp(rint(RN(x_hat / s)), -127, 127); the clamp comes first (rint is monotonic
+            // and +-127 are integers), then adding 1.5 * 2^23 rounds to the nearest even integer
+            // and leaves q in the low byte as two's complement
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+              for (int pi = 0; pi < 4; ++pi) {
+                const bool rb = pi >= 2;
+                float2 qq = make_float2(0.f, 0.f);
+                const float bdiv = rb ? w8_bb : w8_ba;
+                if (bdiv > 0.f) {
+                  const float f = rb ? w8_fb : w8_fa, ny = rb ? w8_nyb : w8_nya;
+                  qq = div_rn2(__fmul2_rn(nx[j][pi], make_float2(f, f)), make_float2(bdiv, bdiv), make_float2(ny, ny));
+                }
+                qq.x = fminf(fmaxf(qq.x, -127.0f), 127.0f);
+                qq.y = fminf(fmaxf(qq.y, -127.0f), 127.0f);
+                qq = __fadd2_rn(qq, make_float2(12582912.0f, 12582912.0f));
+                const uint32_t b2 = (__float_as_uint(qq.x) & 0xFFu) | ((__float_as_uint(qq.y) & 0xFFu) << 8);
+                const int r = rb ? g + 8 : g;
+                const int c = j * 16 + (pi & 1) * 8 + 2 * tig;
+                *reinterpret_cast<uint16_t*>(cst + r * 64 + c) = static_cast<uint16_t>(b2);
+              }
+            }
+          }
         } else {
           if (tig == 0) {
             // 4 consecutive E4M3 bytes of the 128x4 blocked layout per row
@@ -401,16 +457,62 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           }
         }
         __syncwarp();
-        // 16 rows x 32 bytes of codes -> global, one 16-byte segment per lane
-        {
+        if (FMT != kFmtW8a8) {
+          // 16 rows x 32 bytes of codes -> global, one 16-byte segment per lane
           const int r = lane >> 1, h = lane & 1;
           const int row = m0 + strip * 16 + r;
           const uint4 v = *reinterpret_cast<const uint4*>(cst + r * 32 + h * 16);
           if (row < p.M) *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * K2 + col0 / 2 + h * 16) = v;
+        } else if (pass == 1) {
+          // 16 rows x 64 bytes of 8-bit codes -> global, two 16-byte segments per lane
+          const int r = lane >> 1, h = lane & 1;
+          const int row = m0 + strip * 16 + r;
+          const uint4 v0 = *reinterpret_cast<const uint4*>(cst + r * 64 + h * 32);
+          const uint4 v1 = *reinterpret_cast<const uint4*>(cst + r * 64 + h * 32 + 16);
+          if (row < p.M) {
+            uint8_t* dst = p.codes + static_cast<size_t>(row) * p.K + col0 + h * 32;
+            *reinterpret_cast<uint4*>(dst) = v0;
+            *reinterpret_cast<uint4*>(dst + 16) = v1;
+          }
         }
         __syncwarp();
       }
       if (lane == 0) ptx::mbar_arrive(&empty[s]);
+    }
+    if (FMT == kFmtW8a8 && pass == 0) {
+      // Row maxima of the whole K: quad lanes, then the BOXES warps of each row strip.  Every
+      // compute warp reaches this barrier (a wait that ran out only ends the loop above).
+      rmax_a = fmaxf(rmax_a, __shfl_xor_sync(0xffffffffu, rmax_a, 1));
+      rmax_b = fmaxf(rmax_b, __shfl_xor_sync(0xffffffffu, rmax_b, 1));
+      rmax_a = fmaxf(rmax_a, __shfl_xor_sync(0xffffffffu, rmax_a, 2));
+      rmax_b = fmaxf(rmax_b, __shfl_xor_sync(0xffffffffu, rmax_b, 2));
+      if (tig == 0) {
+        rmax_s[(phase * 2 + strip) * 16 + g] = rmax_a;
+        rmax_s[(phase * 2 + strip) * 16 + g + 8] = rmax_b;
+      }
+      named_barrier_sync(2, 32 * NW);
+      float amax_a = 0.f, amax_b = 0.f;
+#pragma unroll
+      for (int ph2 = 0; ph2 < BOXES; ++ph2) {
+        amax_a = fmaxf(amax_a, rmax_s[(ph2 * 2 + strip) * 16 + g]);
+        amax_b = fmaxf(amax_b, rmax_s[(ph2 * 2 + strip) * 16 + g + 8]);
+      }
+      // s = RN_f32(a / 127): the fp64 quotient rounded to fp32 is the correctly rounded fp32
+      // quotient (53 >= 2 * 24 + 2 bits, so the double rounding is innocuous)
+      const float sa = __double2float_rn(__ddiv_rn(static_cast<double>(amax_a), 127.0));
+      const float sb = __double2float_rn(__ddiv_rn(static_cast<double>(amax_b), 127.0));
+      if (phase == 0 && tig == 0) {
+        float* sc = reinterpret_cast<float*>(p.scales);
+        sc[row_a] = sa;             // rows up to Mpad; rows past M read zeros and get 0
+        sc[row_b] = sb;
+      }
+      w8_fa = sa < 0x1p-64f ? 0x1p64f : 1.f;
+      w8_fb = sb < 0x1p-64f ? 0x1p64f : 1.f;
+      w8_ba = sa * w8_fa;            // exact: a power-of-two factor on a tiny scale
+      w8_bb = sb * w8_fb;
+      w8_nya = w8_ba > 0.f ? -__frcp_rn(w8_ba) : 0.f;
+      w8_nyb = w8_bb > 0.f ? -__frcp_rn(w8_bb) : 0.f;
+    }
     }
 
     // ---------------------------------------------------------------- Z = X_hat L1^T
@@ -450,18 +552,19 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   }
 }
 
-template <int RANK>
+template <int FMT, int RANK>
 size_t smem_bytes_for(int stages) {
   constexpr int NW = compute_warps(RANK);
   const ProSmemLayout L = pro_layout(RANK, NW / 2);
-  return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + NW * 512 + 16;
+  return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + NW * code_stage_bytes(FMT) +
+         (NW / 2) * 32 * 4 + 16;
 }
 
-template <int RANK>
+template <int FMT, int RANK>
 int stages_for() {
   constexpr int NW = compute_warps(RANK);
   const ProSmemLayout L = pro_layout(RANK, NW / 2);
-  const size_t budget = 220 * 1024 - 1024 - NW * 512 - 64;
+  const size_t budget = 220 * 1024 - 1024 - NW * code_stage_bytes(FMT) - (NW / 2) * 32 * 4 - 64;
   int s = static_cast<int>(budget / L.stage_bytes);
   if (s > 4) s = 4;
   return s;
@@ -469,9 +572,9 @@ int stages_for() {
 
 template <int FMT, int RANK>
 static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, ProParams p, cudaStream_t stream) {
-  p.stages = stages_for<RANK>();
+  p.stages = stages_for<FMT, RANK>();
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
-  const size_t smem = smem_bytes_for<RANK>(p.stages);
+  const size_t smem = smem_bytes_for<FMT, RANK>(p.stages);
   auto kern = prologue_kernel<FMT, RANK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
@@ -503,6 +606,7 @@ cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& t
                             cudaStream_t s) {
   if (fmt == kFmtNvfp4) return launch_pro_rank<kFmtNvfp4>(tx, tl1, p, s);
   if (fmt == kFmtMxfp4) return launch_pro_rank<kFmtMxfp4>(tx, tl1, p, s);
+  if (fmt == kFmtW8a8) return launch_pro_rank<kFmtW8a8>(tx, tl1, p, s);
   return launch_pro_rank<kFmtInt4>(tx, tl1, p, s);
 }
 

@@ -100,6 +100,7 @@ int* device_error_word() {
 size_t scale_bytes(svdq_format fmt, int64_t rows, int64_t K) {
   const int64_t rp = (rows + 127) / 128 * 128;
   if (fmt == SVDQ_FMT_INT4_G64) return static_cast<size_t>(rp * (K / 64) * 2);
+  if (fmt == SVDQ_FMT_W8A8) return static_cast<size_t>(rp * 4);
   return static_cast<size_t>(rp * (K / fp4_group(fmt)));
 }
 
@@ -125,10 +126,10 @@ extern "C" svdq_status svdq_buffer_sizes(svdq_format fmt, int64_t M, int64_t N, 
   if (st != SVDQ_OK) return st;
   if (!out) return SVDQ_ERR_INVALID_ARG;
   out->x = static_cast<size_t>(M * K * 2);
-  out->a_codes = static_cast<size_t>(M * K / 2);
+  out->a_codes = code_bytes(fmt, M, K);
   out->a_scales = scale_bytes(fmt, M, K);
   out->z = static_cast<size_t>(M * rank * 2);
-  out->w_codes = static_cast<size_t>(N * K / 2);
+  out->w_codes = code_bytes(fmt, N, K);
   out->w_scales = scale_bytes(fmt, N, K);
   out->l1 = static_cast<size_t>(int64_t(rank) * K * 2);
   out->l2 = static_cast<size_t>(N * rank * 2);
@@ -209,7 +210,10 @@ extern "C" svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M
   p.Z = static_cast<__nv_bfloat16*>(Z_bf16);
   p.err = device_error_word();
   if (!p.err) return SVDQ_ERR_CUDA;
-  const int kf = fmt == SVDQ_FMT_NVFP4_G16 ? kFmtNvfp4 : (fmt == SVDQ_FMT_MXFP4_G32 ? kFmtMxfp4 : kFmtInt4);
+  const int kf = fmt == SVDQ_FMT_NVFP4_G16   ? kFmtNvfp4
+                 : fmt == SVDQ_FMT_MXFP4_G32 ? kFmtMxfp4
+                 : fmt == SVDQ_FMT_W8A8      ? kFmtW8a8
+                                             : kFmtInt4;
   cudaError_t e = launch_prologue(kf, tx, tl1, p,
                                   static_cast<cudaStream_t>(cuda_stream));
   if (e != cudaSuccess) return cuda_fail(e);
@@ -276,6 +280,22 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
     if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
     e = launch_gemm_fp4(fmt == SVDQ_FMT_MXFP4_G32, ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms,
                         static_cast<cudaStream_t>(cuda_stream));
+  } else if (fmt == SVDQ_FMT_W8A8) {
+    p.tiles_m = static_cast<int>((M + 255) / 256);
+    p.tiles_n = static_cast<int>((N + 255) / 256);
+    p.num_tiles = p.tiles_m * p.tiles_n;
+    CUtensorMap ta, tb, ty;
+    if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, M, 128, 128)) return SVDQ_ERR_CUDA;
+    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K, N, 128, 128)) return SVDQ_ERR_CUDA;
+    if (rank > 0) {
+      if (!make_tmap(&tz, Z_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, M, 64, 128)) return SVDQ_ERR_CUDA;
+      if (!make_tmap(&tl2, L2_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, rank, N, 64, 128)) return SVDQ_ERR_CUDA;
+    } else {
+      tz = ta;
+      tl2 = tb;
+    }
+    if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
+    e = launch_gemm_w8a8(ta, tb, tz, tl2, ty, p, sms, static_cast<cudaStream_t>(cuda_stream));
   } else {
     p.tiles_m = static_cast<int>((M + 127) / 128);
     p.tiles_n = static_cast<int>(N / 128);

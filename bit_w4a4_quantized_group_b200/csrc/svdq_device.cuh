@@ -12,6 +12,7 @@ namespace svdq {
 constexpr int kFmtNvfp4 = 1;
 constexpr int kFmtInt4 = 2;
 constexpr int kFmtMxfp4 = 3;
+constexpr int kFmtW8a8 = 4;
 
 // Codes recorded in the device error word when a bounded wait runs out.
 enum : int {
@@ -25,6 +26,8 @@ enum : int {
   kErrSiteGemmConvFull = 16,
   kErrSiteGemmSfFree = 17,
   kErrSiteGemmSfReady = 18,
+  kErrSiteGemmConvDone = 19,
+  kErrSiteGemmAccFinal = 20,
   kErrSiteSelftest = 90,
 };
 
@@ -54,6 +57,20 @@ __device__ __forceinline__ bool wait_bounded(uint64_t* bar, uint32_t parity, vol
   }
 }
 
+// Tile schedule of the persistent pair GEMMs: cluster c takes the contiguous run
+// [begin, begin + count) of the N-fastest tile numbering, so consecutive tiles of a
+// cluster share the M block.
+struct TileSeq {
+  int begin, count, tiles_n;
+  __device__ TileSeq(int num_tiles, int tiles_n_, int cluster, int nclusters) : tiles_n(tiles_n_) {
+    const int base = num_tiles / nclusters, extra = num_tiles % nclusters;
+    begin = cluster * base + min(cluster, extra);
+    count = base + (cluster < extra ? 1 : 0);
+  }
+  __device__ int mb(int j) const { return (begin + j) / tiles_n; }
+  __device__ int nb(int j) const { return (begin + j) % tiles_n; }
+};
+
 // Named barrier `id` over `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_barrier_sync(int id, int count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
@@ -68,8 +85,8 @@ struct ProParams {
   int M, K, rank, Mpad, stages;
   const float* lam;          // nullable
   float gscale;              // activation tensor scale (NVFP4), 1 for INT4
-  uint8_t* codes;            // [M][K/2]
-  void* scales;              // format-specific layout
+  uint8_t* codes;            // [M][K/2] (W8A8: [M][K])
+  void* scales;              // format-specific layout (W8A8: fp32 [Mpad])
   __nv_bfloat16* Z;          // [M][rank]
   int* err;                  // device error word
 };
@@ -78,10 +95,10 @@ struct GemmParams {
   int M, N, K, rank;
   int Mpad, Npad;
   float out_scale;           // act_gscale * w_gscale
-  const uint8_t* a_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Mpad]
-  const uint8_t* w_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Npad]
-  const uint8_t* a_codes;    // [M][K/2]
-  const uint8_t* w_codes;    // [N][K/2]
+  const uint8_t* a_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Mpad]; W8A8: fp32 [Mpad]
+  const uint8_t* w_scales;   // NVFP4: blocked E4M3; INT4: fp16 [K/64][Npad]; W8A8: fp32 [Npad]
+  const uint8_t* a_codes;    // [M][K/2] (W8A8: s8 [M][K])
+  const uint8_t* w_codes;    // [N][K/2] (W8A8: s8 [N][K])
   const __nv_bfloat16* bias; // nullable
   __nv_bfloat16* Y;          // [M][N]
   int* err;
@@ -96,6 +113,11 @@ cudaError_t launch_gemm_fp4(bool mx, const CUtensorMap& ta, const CUtensorMap& t
                             const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
                             const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
 size_t gemm_int4_smem_bytes();
+// W8A8 GEMM: s32 accumulation of the 8-bit product, per-row / per-column fp32 scales in the
+// epilogue, the low-rank product in a second (fp32) TMEM accumulator.
+cudaError_t launch_gemm_w8a8(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
+                             const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p, int num_sms,
+                             cudaStream_t s);
 cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
                              const CUtensorMap& tl2, const CUtensorMap& ty, const CUtensorMap& tsa,
                              const CUtensorMap& tsb, const GemmParams& p, int num_sms, cudaStream_t s);

@@ -11,7 +11,8 @@ namespace svdq {
 constexpr int kMaxRank = 128;
 
 inline svdq_status check_dims(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank) {
-  if (fmt != SVDQ_FMT_NVFP4_G16 && fmt != SVDQ_FMT_INT4_G64 && fmt != SVDQ_FMT_MXFP4_G32) return SVDQ_ERR_INVALID_ARG;
+  if (fmt != SVDQ_FMT_NVFP4_G16 && fmt != SVDQ_FMT_INT4_G64 && fmt != SVDQ_FMT_MXFP4_G32 && fmt != SVDQ_FMT_W8A8)
+    return SVDQ_ERR_INVALID_ARG;
   if (M < 1 || N < 128 || K < 128) return SVDQ_ERR_INVALID_ARG;
   if (K % 128 != 0 || N % 128 != 0) return SVDQ_ERR_INVALID_ARG;
   if (rank < 0 || rank > kMaxRank || rank % 16 != 0) return SVDQ_ERR_INVALID_ARG;
@@ -36,5 +37,9 @@ bool is_pow2_positive(float g);
 size_t blocked_sf_offset(int64_t row, int64_t grp, int64_t K, int g);
 // Group size of an E2M1 format (16 NVFP4, 32 MXFP4).
 inline int fp4_group(svdq_format fmt) { return fmt == SVDQ_FMT_MXFP4_G32 ? 32 : 16; }
+// Bytes of the codes of `rows` rows: one byte per element for W8A8, half a byte otherwise.
+inline size_t code_bytes(svdq_format fmt, int64_t rows, int64_t K) {
+  return static_cast<size_t>(fmt == SVDQ_FMT_W8A8 ? rows * K : rows * K / 2);
+}
 
 }  // namespace svdq

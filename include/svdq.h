@@ -16,6 +16,7 @@
  *
  * Notation: M = tokens (b), K = input features (m), N = output features (n),
  * r = rank of the low-rank branch.  g = 16 (NVFP4), 32 (MXFP4) or 64 (INT4), G = K / g.
+ * The W8A8 format (8-bit codes, one scale per row) runs through the same two calls.
  *
  * Conventions for every call
  *   - Ownership: the caller owns every buffer.  The library never allocates
@@ -46,6 +47,7 @@
  *                                        byte k/2 when k is even, high nibble when odd.
  *                                        NVFP4, MXFP4: E2M1 code (bit 3 = sign);
  *                                        INT4: 4-bit two's complement in -7..7.
+ *            W8A8: s8 [rows][K]          one byte per element, two's complement in -127..127.
  *   NVFP4 scales  u8 (E4M3), MXFP4 scales u8 (E8M0: the scale is 2^(byte - 127)), both in the
  *       "128x4 blocked" layout, rows padded to Rp = ceil(rows/128)*128:
  *       byte offset of (row, grp) = ((row/128)*(K/(4g)) + grp/4)*512
@@ -53,6 +55,8 @@
  *       size = Rp * K / g bytes.  Padding rows hold 0.
  *   INT4 scales   fp16, group-major, rows padded to Rp = ceil(rows/128)*128:
  *       element offset of (row, grp) = grp*Rp + row;  size = Rp * (K/64) * 2 bytes.
+ *   W8A8 scales   fp32 [Rp], one per row (per token for activations, per output
+ *       channel for weights); size = Rp * 4 bytes.  Padding rows hold 0.
  *   ("rows" is M for activations, N for weights.)
  */
 #ifndef SVDQ_H_
@@ -86,16 +90,23 @@ typedef enum {
    * q = e2m1_satfinite(x / X).  No tensor scale: act_gscale and w_gscale are 1.
    * ("SVDQuant（实验性功能）": its Nunchaku export needs E2M1 weights and activations in
    * 32-element groups, quantized symmetrically.) */
-  SVDQ_FMT_MXFP4_G32 = 3
+  SVDQ_FMT_MXFP4_G32 = 3,
+  /* symmetric INT8 codes -127..127 with one fp32 scale per row spanning all of K:
+   * s = fp32(a/127) with a = max|x| over the row, q = clamp(rint(fp32(x/s)), -127, 127)
+   * (a zero row gives s = 0 and zero codes).  Activations are quantized per token by
+   * the prologue, weights per output channel by the pack.  No tensor scale.
+   * ("SVDQuant 阅读笔记" §8, appendix D: the 8-bit setting uses rank 16, per-token
+   * dynamic activation quantization and per-channel weight quantization.) */
+  SVDQ_FMT_W8A8 = 4
 } svdq_format;
 
 /* Byte sizes of every buffer of one layer call (no allocation happens). */
 typedef struct {
   size_t x;          /* X      M*K*2                */
-  size_t a_codes;    /* M*K/2                       */
+  size_t a_codes;    /* M*K/2 (W8A8: M*K)           */
   size_t a_scales;   /* per the scale layout above  */
   size_t z;          /* M*r*2                       */
-  size_t w_codes;    /* N*K/2                       */
+  size_t w_codes;    /* N*K/2 (W8A8: N*K)           */
   size_t w_scales;   /* per the scale layout above  */
   size_t l1;         /* r*K*2                       */
   size_t l2;         /* N*r*2                       */
@@ -121,12 +132,13 @@ svdq_status svdq_buffer_sizes(svdq_format fmt, int64_t M, int64_t N, int64_t K, 
  *                              q = e2m1_satfinite(fp32(x/(s*g_w)))
  *                       with a = max|x| over the group (a zero scale gives zero codes)
  *                       MXFP4: the rule of SVDQ_FMT_MXFP4_G32 (a zero group gets byte 0)
+ *                       W8A8: the rule of SVDQ_FMT_W8A8, one scale per row of R
  *   *w_gscale           NVFP4: g_w = 2^ceil(log2(max|R| / (6*448))) (1 if R == 0);
- *                       INT4, MXFP4: 1
+ *                       INT4, MXFP4, W8A8: 1
  *   L1_bf16             bf16 of L1 (round to nearest even)
  *   L2_bf16             bf16 of bf16(L2) / (act_gscale * g_w); must be exact
  * act_gscale is the activation tensor scale later given to the device calls
- * (a positive power of two; 1 for INT4 and MXFP4).  Returns SVDQ_ERR_INVALID_ARG for
+ * (a positive power of two; 1 for INT4, MXFP4 and W8A8).  Returns SVDQ_ERR_INVALID_ARG for
  * bad sizes / NULL pointers / a non power-of-two act_gscale, and
  * SVDQ_ERR_UNSUPPORTED if pre-dividing L2 would not be exact in bf16.
  */
@@ -139,7 +151,11 @@ svdq_status svdq_pack_weight(svdq_format fmt, int64_t N, int64_t K, int rank, fl
  * Device prologue ("算法 2" steps 1-3 of "SVDQuant 阅读笔记" §6.1): one read of X.
  *   X_hat = bf16(fp32(X) / lambda)            (IEEE fp32 divide, one bf16 rounding)
  *   a_codes, a_scales = group quantization of X_hat along K (rules of svdq_pack_weight,
- *                       with act_gscale in place of g_w; INT4 and MXFP4 require act_gscale == 1)
+ *                       with act_gscale in place of g_w; INT4, MXFP4 and W8A8 require
+ *                       act_gscale == 1).  W8A8 quantizes each token row with its own
+ *                       scale, so its prologue reads X twice: once for the row maxima
+ *                       (and Z), once to write the codes (the second read is served
+ *                       mostly from L2).
  *   Z = bf16(X_hat L1^T)                      (fp32 accumulation; skipped when rank == 0)
  * X, lambda, L1 are inputs; a_codes, a_scales, Z outputs (Z may be NULL when rank == 0).
  */
@@ -155,6 +171,9 @@ svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M, int64_t K
  * which equals Q(X_hat) Q(R) + Z L2 + bias because L2s = L2 / (act_gscale * w_gscale).
  * The low-rank product is accumulated on the tensor cores into the same fp32
  * accumulator as the 4-bit product, so Y is written exactly once.
+ * W8A8: Y = bf16( s_x[m] s_w[n] sum_k q_x q_w + Z L2^T + bias ), the 8-bit sum exact in
+ * an s32 accumulator and the low-rank product in a second, fp32 accumulator, both on
+ * the tensor cores and combined in the epilogue (act_gscale = w_gscale = 1, L2s = L2).
  * Z and L2s may be NULL when rank == 0; bias may be NULL.
  */
 svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank,

@@ -5,8 +5,8 @@ import torch
 
 from bit_w4a4_quantized_group_b200 import binding as B
 
-from layouts import (bf16_bits_to_f32, blocked_scale_offsets, f32_to_bf16_bits_exact, scales_canonical,
-                     scales_padding, unpack_codes)
+from layouts import (bf16_bits_to_f32, blocked_scale_offsets, codes_canonical, f32_to_bf16_bits_exact,
+                     scales_canonical, scales_padding)
 
 
 def dev_bf16(x: np.ndarray) -> torch.Tensor:
@@ -39,7 +39,7 @@ def run_prologue(fmt, X, lam, gx, L1_rk, fill=0x5A):
     check_device_error()
     sc = scales.cpu().numpy()
     return {
-        "codes": unpack_codes(codes.cpu().numpy(), M, K),
+        "codes": codes_canonical(fmt, codes.cpu().numpy(), M, K),
         "scales": scales_canonical(fmt, sc, M, K),
         "scale_padding": scales_padding(fmt, sc, M, K),
         "Z": host_bf16(Z) if r > 0 else np.zeros((M, 0), np.float32),
@@ -50,6 +50,10 @@ def run_prologue(fmt, X, lam, gx, L1_rk, fill=0x5A):
 def encode_scales(fmt, scale_bits: np.ndarray, rows: int, K: int) -> np.ndarray:
     """Canonical scale bits [rows][G] -> library buffer bytes (padding rows zero)."""
     rp = (rows + 127) // 128 * 128
+    if fmt == "w8a8":
+        buf = np.zeros(rp, np.uint32)
+        buf[:rows] = np.asarray(scale_bits, np.uint32).reshape(rows)
+        return buf.view(np.uint8)
     if fmt in ("nvfp4", "mxfp4"):
         g = 16 if fmt == "nvfp4" else 32
         buf = np.zeros(rp * K // g, np.uint8)
@@ -63,6 +67,13 @@ def encode_scales(fmt, scale_bits: np.ndarray, rows: int, K: int) -> np.ndarray:
 def pack_codes_bytes(codes: np.ndarray) -> np.ndarray:
     c = np.asarray(codes, np.uint8)
     return (c[:, 0::2] | (c[:, 1::2] << 4)).astype(np.uint8).reshape(-1)
+
+
+def codes_bytes(fmt, codes: np.ndarray) -> np.ndarray:
+    """Canonical codes -> library code buffer (nibble pairs, or one byte each for W8A8)."""
+    if fmt == "w8a8":
+        return np.ascontiguousarray(codes, np.uint8).reshape(-1)
+    return pack_codes_bytes(codes)
 
 
 def run_gemm(fmt, M, N, K, rank, a_codes, a_scales, gx, w_codes, w_scales, gw, Z, L2s, bias):

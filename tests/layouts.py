@@ -67,15 +67,37 @@ def int4_scales_padding(buf: np.ndarray, rows: int, K: int) -> np.ndarray:
     return b[:, rows:].copy()
 
 
+def row_scales_canonical(buf, rows: int) -> np.ndarray:
+    """W8A8: fp32 [Rp] -> uint32 bits [rows][1]."""
+    b = np.asarray(buf).reshape(-1).view(np.uint32)
+    return b[:rows].reshape(rows, 1).copy()
+
+
+def row_scales_padding(buf, rows: int) -> np.ndarray:
+    rp = (rows + 127) // 128 * 128
+    return np.asarray(buf).reshape(-1).view(np.uint32)[rows:rp].copy()
+
+
+def codes_canonical(fmt: str, buf, rows: int, K: int) -> np.ndarray:
+    """Codes as the reference returns them: nibbles for the 4-bit formats, bytes for W8A8."""
+    if fmt == "w8a8":
+        return np.asarray(buf, np.uint8).reshape(-1)[: rows * K].reshape(rows, K).copy()
+    return unpack_codes(np.asarray(buf, np.uint8).reshape(-1)[: rows * K // 2], rows, K)
+
+
 def scales_canonical(fmt: str, buf, rows: int, K: int) -> np.ndarray:
     if fmt == "int4":
         return int4_scales_canonical(buf, rows, K)
+    if fmt == "w8a8":
+        return row_scales_canonical(buf, rows)
     return blocked_scales_canonical(buf, rows, K, 16 if fmt == "nvfp4" else 32)
 
 
 def scales_padding(fmt: str, buf, rows: int, K: int) -> np.ndarray:
     if fmt == "int4":
         return int4_scales_padding(buf, rows, K)
+    if fmt == "w8a8":
+        return row_scales_padding(buf, rows)
     return blocked_scales_padding(buf, rows, K, 16 if fmt == "nvfp4" else 32)
 
 

@@ -16,7 +16,8 @@ from bit_w4a4_quantized_group_b200 import binding as B
 from bit_w4a4_quantized_group_b200 import build as BUILD
 from bit_w4a4_quantized_group_b200 import inputs as I
 
-from layouts import int4_scales_canonical, nvfp4_scales_canonical, scales_canonical, scales_padding, unpack_codes
+from layouts import (codes_canonical, int4_scales_canonical, nvfp4_scales_canonical, scales_canonical, scales_padding,
+                     unpack_codes)
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -50,6 +51,10 @@ def test_buffer_sizes(lib):
     assert s.y == 300 * 640 * 2 and s.bias == 640 * 2
     s = B.svdq_buffer_sizes("int4", 300, 640, 768, 0)
     assert s.a_scales == 384 * (768 // 64) * 2 and s.z == 0
+    s = B.svdq_buffer_sizes("w8a8", 300, 640, 768, 16)
+    assert s.a_codes == 300 * 768 and s.w_codes == 640 * 768
+    assert s.a_scales == 384 * 4 and s.w_scales == 640 * 4
+    assert s.z == 300 * 16 * 2 and s.l2 == 640 * 16 * 2
 
 
 @pytest.mark.parametrize("args", [
@@ -120,7 +125,7 @@ def _check_pack(fmt, R_nk, L1_rk, L2_nr, gx):
     got = B.pack_weight_np(fmt, R_nk, L1_rk, L2_nr, gx)
     ref = O.pack_weight(fmt, R_nk, L1_rk, L2_nr, gx)
     assert got["w_gscale"] == ref["gscale"]
-    assert np.array_equal(unpack_codes(got["w_codes"], N, K), ref["q"]["codes"])
+    assert np.array_equal(codes_canonical(fmt, got["w_codes"], N, K), ref["q"]["codes"])
     assert np.array_equal(scales_canonical(fmt, got["w_scales"], N, K), ref["q"]["scale_bits"])
     assert np.all(scales_padding(fmt, got["w_scales"], N, K) == 0)
     if L1_rk is not None and L1_rk.shape[0] > 0:
@@ -130,7 +135,7 @@ def _check_pack(fmt, R_nk, L1_rk, L2_nr, gx):
         assert np.array_equal(l2, ref["L2_scaled"])
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 def test_pack_weight_matches_reference_on_tiny_layer(lib, fmt):
     layer = I.make_layer(I.TINY)
     prep = O.prepare_layer(fmt, layer.X, layer.W, 16)
@@ -138,7 +143,7 @@ def test_pack_weight_matches_reference_on_tiny_layer(lib, fmt):
                 prep["act_gscale"])
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("scale_exp", [-12, -3, 0, 6])
 def test_pack_weight_matches_reference_random(lib, fmt, scale_exp):
     rng = np.random.default_rng(100 + scale_exp)
@@ -174,6 +179,14 @@ def test_pack_weight_rank0_and_ties(lib):
     R3[:, 32] = 2.0 ** -140
     R3[:, 64] = -0.0
     _check_pack("mxfp4", R3, None, None, 1.0)
+    # W8A8: max 127 gives s = 1 and the midpoints round to even; a tiny row has a subnormal scale
+    R4 = np.zeros((N, K), np.float32)
+    R4[:, 0] = 127.0
+    R4[:, 1:7] = [0.5, 1.5, 2.5, -0.5, -126.5, 0.49]
+    R4[5, :] = 0.0
+    R4[6, :3] = [1e-40, -3e-41, 7e-42]
+    R4[7, :] = -0.0
+    _check_pack("w8a8", R4, None, None, 1.0)
 
 
 def test_pack_weight_rejects(lib):
@@ -185,6 +198,8 @@ def test_pack_weight_rejects(lib):
         B.pack_weight_np("int4", R, None, None, 0.5)      # INT4 needs g_x = 1
     with pytest.raises(B.SvdqError):
         B.pack_weight_np("mxfp4", R, None, None, 2.0)     # MXFP4 has no tensor scale
+    with pytest.raises(B.SvdqError):
+        B.pack_weight_np("w8a8", R, None, None, 2.0)      # nor has W8A8
 
 
 def test_selftest_rejects_limits_out_of_range():

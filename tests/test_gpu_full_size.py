@@ -24,7 +24,7 @@ from bit_w4a4_quantized_group_b200 import inputs as I
 from bit_w4a4_quantized_group_b200.layer import W4A4LowRankLinear
 
 from gpu_helpers import assert_y_elementwise, check_device_error, dev_bf16, host_bf16, rel_fro, y_elementwise_slack
-from layouts import bf16_ulp, scales_canonical, unpack_codes
+from layouts import bf16_ulp, codes_canonical, scales_canonical
 
 pytestmark = pytest.mark.gpu
 
@@ -65,7 +65,7 @@ def _run_and_check(cfg, fmt, rows=None, seed=4242):
     if rows is None:
         rows = np.arange(M)
     ws = lin.workspace(M)
-    codes = unpack_codes(ws["a_codes"].cpu().numpy(), M, K)[rows]
+    codes = codes_canonical(fmt, ws["a_codes"].cpu().numpy(), M, K)[rows]
     scales = scales_canonical(fmt, ws["a_scales"].cpu().numpy(), M, K)[rows]
     Yall = host_bf16(Y)
     assert np.all(np.isfinite(Yall))
@@ -103,6 +103,13 @@ def _sample_rows(M, seed):
 def test_full_size_layer_sampled_rows(name, fmt):
     cfg = I.NAMED[name]
     _run_and_check(cfg, fmt, _sample_rows(cfg.b, 7))
+
+
+@pytest.mark.parametrize("name", ["mlp_up", "mlp_down", "qkv"])
+def test_full_size_w8a8_rank16_sampled_rows(name):
+    """The 8-bit setting (per-token activations, per-channel weights, rank 16) at full size."""
+    cfg = dataclasses.replace(I.NAMED[name], rank=16)
+    _run_and_check(cfg, "w8a8", _sample_rows(cfg.b, 8))
 
 
 def test_sweep_largest_batch_sampled_rows():

@@ -16,7 +16,7 @@ from bit_w4a4_quantized_group_b200 import binding as B
 from bit_w4a4_quantized_group_b200 import build as BUILD
 from bit_w4a4_quantized_group_b200 import inputs as I
 
-from gpu_helpers import (assert_y_elementwise, encode_scales, host_bf16, pack_codes_bytes, rel_fro, run_gemm,
+from gpu_helpers import (assert_y_elementwise, codes_bytes, encode_scales, host_bf16, rel_fro, run_gemm,
                          run_prologue, y_elementwise_slack)
 from layouts import bf16_ulp
 
@@ -61,7 +61,7 @@ def _check_prologue(fmt, X, lam, gx, L1_rk):
     return got, ref
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
                                       (96, 512, 128)])
 def test_prologue_parity(fmt, M, K, rank):
@@ -69,7 +69,7 @@ def test_prologue_parity(fmt, M, K, rank):
     _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 def test_prologue_without_smoothing_and_zero_rows(fmt):
     rng = np.random.default_rng(5)
     X = I.to_bf16(rng.standard_normal((200, 384)) * 3)
@@ -113,6 +113,29 @@ def test_prologue_rounding_mxfp4_scales_ties_and_saturation():
     _check_prologue("mxfp4", X, None, 1.0, None)
 
 
+def test_prologue_rounding_w8a8_rows():
+    """W8A8 per-token rows: max 127 (s = 1) with midpoints that round to even, a row whose
+    maximum sits in the last K stage, a zero row (s = 0, zero codes), a row small enough that
+    the divide takes the power-of-two prescale (s < 2^-64), a subnormal-scale row and a row
+    near the bf16 maximum; K spans several stages and M leaves padding rows."""
+    M, K = 200, 1280
+    X = np.zeros((M, K), np.float32)
+    X[:, 0] = 127.0
+    X[:, 1:9] = [0.5, 1.5, 2.5, -0.5, -126.5, 63.5, 0.49609375, -3.5]
+    X[1, 0] = 1.0
+    X[1, K - 1] = -300.0                                 # the row maximum in the last stage
+    X[2:6] = 0.0                                         # zero row (2); rows 3-5 start empty
+    X[3, :4] = [2.0 ** -70, -3.0 * 2.0 ** -72, 2.0 ** -80, 0.0]   # s < 2^-64
+    X[4, :3] = [2.0 ** -125, -2.0 ** -127, 2.0 ** -133]            # subnormal scale
+    X[5, :3] = [3.0e38, -1.0e38, 1.0]
+    rng = np.random.default_rng(41)
+    X[6:] = rng.standard_normal((M - 6, K)) * np.exp2(rng.integers(-8, 8, (M - 6, 1)))
+    X = I.to_bf16(X)
+    got, ref = _check_prologue("w8a8", X, None, 1.0, None)
+    assert list(got["codes"][0, :9].view(np.int8)) == [127, 0, 2, 2, 0, -126, 64, 0, -4]
+    assert got["scales"][2, 0] == 0 and np.all(got["codes"][2] == 0)
+
+
 def test_prologue_rounding_ties_int4():
     M, K = 128, 128
     X = np.zeros((M, K), np.float32)
@@ -130,8 +153,8 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     bias = layer.bias if with_bias else None
     ref = O.gemm_forward(pro["q"], gx, packed["q"], packed["gscale"], pro["Z"], packed["L2_bf16"], bias)
     Y = run_gemm(fmt, M, N, K, rank,
-                 pack_codes_bytes(pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
-                 pack_codes_bytes(packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
+                 codes_bytes(fmt, pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
+                 codes_bytes(fmt, packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
                  packed["gscale"], pro["Z"], packed["L2_scaled"], bias)
     Yg = host_bf16(Y)
     assert np.all(np.isfinite(Yg))
@@ -144,14 +167,14 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     return Yg, ref
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,N,K,rank", [(300, 640, 640, 32), (256, 512, 512, 16), (128, 256, 256, 0),
                                         (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64)])
 def test_gemm_parity(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=11 + M + N + rank)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,N,K,rank", [(2304, 3072, 512, 32), (2560, 2560, 256, 0), (2304, 3072, 256, 128),
                                         (1300, 3072, 768, 16)])
 def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
@@ -160,12 +183,12 @@ def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=5 + M + K + rank)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 def test_gemm_parity_no_bias(fmt):
     _gemm_case(fmt, 160, 512, 512, 32, seed=3, with_bias=False)
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 def test_gemm_lowrank_branch_is_added(fmt):
     """Y(r) - Y(r=0 on the same 4-bit operands) equals Z L2 (the branch really lands in Y)."""
     M, N, K, rank = 128, 256, 256, 32
@@ -173,8 +196,8 @@ def test_gemm_lowrank_branch_is_added(fmt):
     gx = prep["act_gscale"]
     packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
     pro = O.prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"])
-    args = (pack_codes_bytes(pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
-            pack_codes_bytes(packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
+    args = (codes_bytes(fmt, pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
+            codes_bytes(fmt, packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
             packed["gscale"])
     Y1 = host_bf16(run_gemm(fmt, M, N, K, rank, *args, pro["Z"], packed["L2_scaled"], None)).astype(np.float64)
     Y0 = host_bf16(run_gemm(fmt, M, N, K, 0, *args, None, None, None)).astype(np.float64)
@@ -183,7 +206,8 @@ def test_gemm_lowrank_branch_is_added(fmt):
 
 
 @pytest.mark.parametrize("fmt,rank", [("nvfp4", 32), ("nvfp4", 0), ("nvfp4", 128), ("int4", 32), ("int4", 0),
-                                      ("int4", 128), ("mxfp4", 32), ("mxfp4", 0), ("mxfp4", 128)])
+                                      ("int4", 128), ("mxfp4", 32), ("mxfp4", 0), ("mxfp4", 128),
+                                      ("w8a8", 16), ("w8a8", 0), ("w8a8", 128)])
 def test_layer_end_to_end_small(fmt, rank):
     """Prologue then GEMM on the device (Z never leaves the GPU) vs the reference layer."""
     M, K, N = 384, 768, 768
