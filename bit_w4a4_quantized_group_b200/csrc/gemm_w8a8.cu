@@ -18,8 +18,8 @@
 //     run while the epilogue drains tile t;
 //   * the branch cannot share the s32 accumulator, so the epilogue first converts it in
 //     place: acc -> fp32(acc) * s_x s_w, written back with tcgen05.st.  The MMA warp then
-//     adds Z L2^T onto the converted values with kind::f16 MMAs (accumulate on), issued a
-//     few steps into the next tile's main loop so that the conversion has finished by then
+//     adds Z L2^T onto the converted values with kind::f16 MMAs (accumulate on), issued
+//     halfway through the next tile's main loop so that the conversion has finished by then
 //     and the tensor pipe does not wait for it;
 //   * eight epilogue warps per CTA read the final fp32 values, add the bias and store bf16
 //     Y through 128B-swizzled staging and TMA stores.
@@ -46,7 +46,6 @@ constexpr uint32_t kStageBytes = kABytes + kBBytes;
 constexpr uint32_t kTx = 2 * kStageBytes;     // both CTAs (main and low-rank steps alike)
 constexpr uint32_t kEpiBoxBytes = 32 * 128;   // 32 rows x 64 bf16 per epilogue warp
 constexpr uint32_t kTmemCols = 512;           // two accumulators of 256 columns
-constexpr int kLrAt = 4;                      // branch of tile t-1 issued after this many steps of tile t
 
 __host__ __device__ constexpr uint32_t idesc_s8(int m, int n) {
   // s8 x s8 -> s32, K-major A and B
@@ -71,8 +70,10 @@ struct SharedTail {
 };
 
 // Position of the low-rank steps in the pipeline: those of tile t-1 come after the first
-// `ins` main steps of tile t; those of the last tile come after its main steps.
-__device__ __forceinline__ int lr_insert_at(int nk_main) { return nk_main < kLrAt ? nk_main : kLrAt; }
+// `ins` main steps of tile t (half of them: by then the epilogue has long finished converting
+// tile t-1, while the epilogue still has the other half to read tile t-1's final values before
+// tile t+1 needs the buffer); those of the last tile come after its main steps.
+__device__ __forceinline__ int lr_insert_at(int nk_main) { return nk_main > 1 ? nk_main / 2 : 1; }
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_w8a8_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
