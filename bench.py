@@ -58,6 +58,9 @@ def parse_args():
                          "the kernels' time and traffic do not depend on the weight values)")
     ap.add_argument("--residual-iters", type=int, default=1,
                     help="outer residual iterations of the offline split (1: plain SVD split)")
+    ap.add_argument("--sweep", action="store_true",
+                    help="instead of the headline line, time the layer over the batch x shape x rank grid "
+                         "(random weights of each shape) and print one JSON line per point")
     ap.add_argument("--residual-early-stop", action="store_true",
                     help="keep the best residual-iteration candidate and stop once the target gets worse")
     return ap.parse_args()
@@ -346,10 +349,100 @@ def config_dict(cfg, fmt, l2):
 
 # ----------------------------------------------------------------------------- GPU path
 
+def run_sweep(args):
+    """Layer time over the batch x shape x rank grid, one JSON line per point.
+
+    Each point uses seeded random weights of its shape (kernel time does not depend on the
+    values), the fused layer (prologue + GEMM), the same layer at rank 0 and the unfused
+    branch (separate passes on cuBLAS bf16) on top of the rank-0 layer.  L2 is flushed
+    between timed calls.
+    """
+    import torch
+    from bit_w4a4_quantized_group_b200 import binding as B
+    from bit_w4a4_quantized_group_b200 import build as BUILD
+    from bit_w4a4_quantized_group_b200 import inputs as I
+    from bit_w4a4_quantized_group_b200 import prepare as P
+    from bit_w4a4_quantized_group_b200.layer import W4A4LowRankLinear
+    from bit_w4a4_quantized_group_b200.inputs import bf16_bits
+    if int(os.environ.get("RANK", "0")) != 0:
+        return 0
+    BUILD.build()
+    B.load()
+    device = torch.device("cuda", int(os.environ.get("LOCAL_RANK", "0")))
+    torch.cuda.set_device(device)
+    fmt = args.format
+    stream = torch.cuda.current_stream()
+    flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
+    bf16_burst, _, _, _ = peaks()
+    peak = bf16_burst * (4.0 if fmt in ("nvfp4", "mxfp4") else 2.0)
+
+    def timed(fn, n):
+        for _ in range(args.warmup):
+            flush.zero_()
+            fn()
+        evs = []
+        for _ in range(n):
+            flush.zero_()
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            evs.append((a, b))
+        torch.cuda.synchronize()
+        return sum(a.elapsed_time(b) for a, b in evs) / n * 1e-3
+
+    for cfg in I.sweep_configs():
+        layer = I.make_layer(cfg)
+        M, K, N, r = cfg.b, cfg.m, cfg.n, cfg.rank
+        rng = np.random.default_rng(cfg.seed + 1000)
+        xa = float(np.abs(layer.X).max())
+        prep = {"lam": np.ones(K, np.float32),
+                "R_nk": (rng.standard_normal((N, K)) * cfg.sigma_w).astype(np.float32),
+                "L1_rk": (rng.standard_normal((r, K)) * 0.05).astype(np.float32),
+                "L2_nr": (rng.standard_normal((N, r)) * 0.05).astype(np.float32),
+                "act_gscale": P.pow2_tensor_scale(xa) if fmt == "nvfp4" else 1.0}
+        lin = W4A4LowRankLinear(fmt, N, K, P.pack(fmt, prep), prep["lam"], prep["act_gscale"], layer.bias,
+                                device=device)
+        X = torch.from_numpy(bf16_bits(layer.X).view(np.int16)).to(device).view(torch.bfloat16)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        n = max(5, args.steps)
+        t_layer = timed(lambda: lin.forward(X, Y), n)
+        t_pro = timed(lambda: lin.prologue_only(X), n)
+        t_gemm = timed(lambda: lin.gemm_only(M, Y), n)
+        t_r0 = timed(lambda: (lin.prologue_only(X, rank=0), lin.gemm_only(M, Y, rank=0)), n)
+        out = {"sweep_point": cfg.name, "format": fmt, "M": M, "K": K, "N": N, "rank": r,
+               "lora_rank": cfg.lora_rank, "layer_us": t_layer * 1e6, "prologue_us": t_pro * 1e6,
+               "gemm_us": t_gemm * 1e6, "tflops": 2.0 * M * N * K / t_layer / 1e12,
+               "gemm_frac": (2.0 * M * N * K + 2.0 * M * N * r) / t_gemm / 1e12 / peak,
+               "layer_r0_us": t_r0 * 1e6, "fused_overhead_pct": 100.0 * (t_layer / t_r0 - 1.0)}
+        if r > 0:
+            up_scale = lin.act_gscale * lin.w_gscale
+            lam_d = torch.ones(K, device=device)
+
+            def unfused():
+                lin.prologue_only(X, rank=0)
+                lin.gemm_only(M, Y, rank=0)
+                xh = (X.float() / lam_d).to(torch.bfloat16)
+                Y.addmm_(xh @ lin.L1.t(), lin.L2.t(), alpha=up_scale)
+            t_unf = timed(unfused, n)
+            out["unfused_layer_us"] = t_unf * 1e6
+            out["unfused_overhead_pct"] = 100.0 * (t_unf / t_r0 - 1.0)
+        st, site = B.svdq_get_last_device_error(None)
+        if st != B.SVDQ_OK:
+            raise RuntimeError(f"device error {st} at site {site}")
+        print(json.dumps(out), flush=True)
+        del lin, X, Y
+        torch.cuda.empty_cache()
+    return 0
+
+
 def main():
     args = parse_args()
     if args.impl == "reference":
         return run_reference(args)
+    if args.sweep:
+        return run_sweep(args)
 
     import torch
     import torch.distributed as dist
@@ -422,6 +515,22 @@ def main():
     t_pro = sum(e[0].elapsed_time(e[1]) for e in ev) / args.steps * 1e-3
     t_gemm = sum(e[1].elapsed_time(e[2]) for e in ev) / args.steps * 1e-3
     t_step = t_pro + t_gemm
+    steps_us = sorted(e[0].elapsed_time(e[2]) * 1e3 for e in ev)
+
+    def pct(q):
+        return steps_us[min(len(steps_us) - 1, int(round(q * (len(steps_us) - 1))))]
+    step_dist = {"p10": pct(0.1), "p50": pct(0.5), "p90": pct(0.9)}
+    # the same step with a warm L2 (no flush in between): reported beside the headline only
+    hot = []
+    for i in range(max(5, args.steps // 2)):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        lin.forward(X, Y)
+        b.record(stream)
+        hot.append((a, b))
+    torch.cuda.synchronize()
+    t_hot = sum(a.elapsed_time(b) for a, b in hot) / len(hot) * 1e-3
 
     # low-rank overhead: the same GEMM without the branch (not part of the headline)
     gemm0 = []
@@ -554,6 +663,8 @@ def main():
             "unfused_vs_fused_rel_fro": fusion["rel"]},
         "gpu_launches": launches,
         "clocks": clk,
+        "step_us": step_dist,
+        "hot_l2_ms_per_step": t_hot * 1e3,
     }
     if "offline_s" in prep:
         res = prep.get("residual") or {}
