@@ -64,7 +64,8 @@ def qdq_weight(fmt: str, R_nk: torch.Tensor) -> torch.Tensor:
     INT4 g64: s = fp16(fp32(a / 7)) (clamped to 65504), q = rint(fp32(R / s)) in [-7, 7].
     NVFP4 g16: s = e4m3(fp32(fp32(a / 6) / g_w)) with g_w the power-of-two tensor scale,
     q = e2m1(fp32(R / fp32(s g_w))).  MXFP4 g32: X = 2^clip(floor(log2 a) - 2, -127, 127),
-    q = e2m1(R / X).  Returns g s q in fp64.
+    q = e2m1(R / X).  W8A8: one scale per row, s = fp32(a / 127), q = clamp(rint(fp32(R / s)),
+    -127, 127).  Returns g s q in fp64.
     """
     R = R_nk.to(torch.float32)
     N, K = R.shape
@@ -86,6 +87,12 @@ def qdq_weight(fmt: str, R_nk: torch.Tensor) -> torch.Tensor:
         q = _e2m1_rn(Rg / safe[..., None])
         q = torch.where((den > 0)[..., None], q, torch.zeros_like(q))
         return (q * den.to(torch.float64)[..., None]).reshape(N, K)
+    if fmt == "w8a8":
+        s = R.abs().amax(1, keepdim=True) / 127.0
+        safe = torch.where(s > 0, s, torch.ones_like(s))
+        q = torch.clamp(torch.round(R / safe), -127.0, 127.0)
+        q = torch.where(s > 0, q, torch.zeros_like(q))
+        return q.to(torch.float64) * s.to(torch.float64)
     if fmt == "mxfp4":
         Rg = R.reshape(N, K // 32, 32)
         a = Rg.abs().amax(2).to(torch.float64)

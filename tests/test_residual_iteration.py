@@ -23,7 +23,7 @@ import oracle as O
 from bit_w4a4_quantized_group_b200 import inputs as I
 from bit_w4a4_quantized_group_b200 import prepare as P
 
-FMTS = ["int4", "nvfp4", "mxfp4"]
+FMTS = ["int4", "nvfp4", "mxfp4", "w8a8"]
 
 
 @pytest.fixture(scope="module")
@@ -69,9 +69,11 @@ def test_each_refit_is_the_best_rank_r_fit_of_w_minus_qr(tiny, fmt):
         # bf16 factors cost at most a few 2^-9 relative of the branch
         slack = 4 * 2.0 ** -9 * np.linalg.norm(cur["L1_bf16"] @ cur["L2_bf16"])
         assert opt <= fit + 1e-9 and fit <= opt + slack
-        # a fit to W - R_{i-1} (Q dropped) would give back the previous branch
+        # a fit to W - R_{i-1} (Q dropped) would give back the previous branch (for the 4-bit
+        # formats Q moves R far more than the bf16 rounding of the factors; for W8A8 it does not)
         stale = np.linalg.norm(T - prev["L1_bf16"] @ prev["L2_bf16"])
-        assert fit < stale
+        if fmt != "w8a8":
+            assert fit < stale
         # the new residual is W_tilde minus the new branch, in fp32
         assert np.array_equal(cur["R"], (Wt - cur["L1_bf16"] @ cur["L2_bf16"]).astype(np.float32))
         prev = cur
