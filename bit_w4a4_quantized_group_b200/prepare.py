@@ -69,9 +69,14 @@ def qdq_weight(fmt: str, R_nk: torch.Tensor) -> torch.Tensor:
     """
     R = R_nk.to(torch.float32)
     N, K = R.shape
+
+    def div(x: torch.Tensor, c: float) -> torch.Tensor:
+        # a tensor divisor keeps the IEEE divide (a Python-scalar divisor may become a
+        # multiply by its reciprocal on the device, which is not the same rounding)
+        return x / torch.full_like(x, c)
     if fmt == "int4":
         Rg = R.reshape(N, K // 64, 64)
-        t = Rg.abs().amax(2) / 7.0
+        t = div(Rg.abs().amax(2), 7.0)
         s = torch.clamp(t.to(torch.float16).to(torch.float32), max=65504.0)
         safe = torch.where(s > 0, s, torch.ones_like(s))
         q = torch.clamp(torch.round(Rg / safe[..., None]), -7.0, 7.0)
@@ -80,7 +85,7 @@ def qdq_weight(fmt: str, R_nk: torch.Tensor) -> torch.Tensor:
     if fmt == "nvfp4":
         gw = pow2_tensor_scale(float(R.abs().max())) if R.numel() else 1.0
         Rg = R.reshape(N, K // 16, 16)
-        t = (Rg.abs().amax(2) / 6.0) / gw
+        t = div(div(Rg.abs().amax(2), 6.0), gw)
         s = torch.clamp(t, max=448.0).to(torch.float8_e4m3fn).to(torch.float32)
         den = s * gw
         safe = torch.where(den > 0, den, torch.ones_like(den))
@@ -88,7 +93,7 @@ def qdq_weight(fmt: str, R_nk: torch.Tensor) -> torch.Tensor:
         q = torch.where((den > 0)[..., None], q, torch.zeros_like(q))
         return (q * den.to(torch.float64)[..., None]).reshape(N, K)
     if fmt == "w8a8":
-        s = R.abs().amax(1, keepdim=True) / 127.0
+        s = div(R.abs().amax(1, keepdim=True), 127.0)
         safe = torch.where(s > 0, s, torch.ones_like(s))
         q = torch.clamp(torch.round(R / safe), -127.0, 127.0)
         q = torch.where(s > 0, q, torch.zeros_like(q))
