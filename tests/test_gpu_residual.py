@@ -19,7 +19,7 @@ from bit_w4a4_quantized_group_b200 import prepare as P
 from bit_w4a4_quantized_group_b200.layer import W4A4LowRankLinear
 
 from gpu_helpers import assert_y_elementwise, check_device_error, dev_bf16, host_bf16, rel_fro, y_elementwise_slack
-from layouts import scales_canonical, unpack_codes
+from layouts import codes_canonical, scales_canonical
 from test_residual_iteration import FMTS, _deployed_qdq, _qdq_cases
 
 pytestmark = pytest.mark.gpu
@@ -75,7 +75,7 @@ def test_layer_from_iterated_split_runs_at_parity(fmt):
     ws = lin.workspace(M)
     packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
     pro = O.prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"])
-    np.testing.assert_array_equal(unpack_codes(ws["a_codes"].cpu().numpy(), M, K), pro["q"]["codes"])
+    np.testing.assert_array_equal(codes_canonical(fmt, ws["a_codes"].cpu().numpy(), M, K), pro["q"]["codes"])
     np.testing.assert_array_equal(scales_canonical(fmt, ws["a_scales"].cpu().numpy(), M, K), pro["q"]["scale_bits"])
     Zg = host_bf16(ws["Z"])
     Yg = host_bf16(Y)
