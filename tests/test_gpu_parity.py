@@ -288,3 +288,34 @@ def test_tiny_layer_int4_end_to_end():
     assert rel_fro(Yg, ref_gz["Y"]) <= Y_TOL
     exact = layer.X.astype(np.float64) @ layer.W + layer.bias.astype(np.float64)
     assert rel_fro(Yg, exact) < 0.15
+
+
+def _bf16_values_up_to(bound):
+    """Every finite bf16 value v with |v| <= bound (both signs, zeros and subnormals included)."""
+    bits = np.arange(65536, dtype=np.uint32)
+    v = (bits << 16).view(np.float32)
+    return v[np.isfinite(v) & (np.abs(v) <= bound)]
+
+
+@pytest.mark.parametrize("fmt,gmax", [("nvfp4", 6.0), ("nvfp4", 6.75), ("nvfp4", 2688.0), ("mxfp4", 7.5),
+                                      ("mxfp4", 6.0 * 2.0 ** -20), ("int4", 7.0), ("int4", 7.75),
+                                      ("w8a8", 127.0), ("w8a8", 100.5)])
+def test_prologue_codes_exhaustive_over_bf16(fmt, gmax):
+    """The quantizer's input is a bf16 X_hat, so every bf16 value under a group's (or row's)
+    maximum is the whole input space for that scale: each group holds the maximum in its
+    first slot and a run of the sweep in the others; codes and scales must match the
+    reference bit for bit (unit scales, scales with more mantissa bits, saturation)."""
+    g = {"nvfp4": 16, "mxfp4": 32, "int4": 64, "w8a8": 128}[fmt]
+    K = 128
+    vals = _bf16_values_up_to(gmax)
+    per_group = g - 1
+    ngroups = -(-len(vals) // per_group)
+    pad = np.zeros(ngroups * per_group, np.float32)
+    pad[: len(vals)] = vals
+    grp = np.concatenate([np.full((ngroups, 1), gmax, np.float32), pad.reshape(ngroups, per_group)], axis=1)
+    rows = -(-ngroups // (K // g))
+    allg = np.zeros((rows * (K // g), g), np.float32)
+    allg[:ngroups] = grp
+    X = I.to_bf16(allg.reshape(rows, K))
+    assert np.array_equal(X, allg.reshape(rows, K))           # every value is already bf16
+    _check_prologue(fmt, X, None, 1.0, None)
