@@ -206,3 +206,34 @@ def test_selftest_rejects_limits_out_of_range():
     # argument checks run before any CUDA call
     assert B.svdq_selftest_bounded_wait(10, None) == B.SVDQ_ERR_INVALID_ARG
     assert B.svdq_selftest_bounded_wait(10_000_000_000, None) == B.SVDQ_ERR_INVALID_ARG
+
+
+# ------------------------------------------------------- randomized host pack parity
+
+from hypothesis import HealthCheck, given, settings
+from hypothesis import strategies as st
+
+
+@settings(max_examples=30, deadline=None, suppress_health_check=[HealthCheck.function_scoped_fixture])
+@given(fmt=st.sampled_from(["nvfp4", "int4", "mxfp4", "w8a8"]),
+       nb=st.integers(1, 3), kb=st.integers(1, 4), rank=st.sampled_from([0, 16, 32]),
+       exp=st.integers(-30, 20), dist=st.sampled_from(["normal", "heavy", "uniform", "sparse"]),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_pack_weight_matches_reference_randomized(lib, fmt, nb, kb, rank, exp, dist, seed):
+    """Shapes, magnitudes and distributions drawn at random; codes, scales, g_w and the
+    factors must match the CPU reference bit for bit."""
+    rng = np.random.default_rng(seed)
+    N, K = 128 * nb, 128 * kb
+    if dist == "normal":
+        R = rng.standard_normal((N, K))
+    elif dist == "heavy":
+        R = rng.standard_t(2.0, (N, K))
+    elif dist == "uniform":
+        R = rng.uniform(-1, 1, (N, K))
+    else:
+        R = rng.standard_normal((N, K)) * (rng.random((N, K)) < 0.05)
+    R = (R * 2.0 ** exp).astype(np.float32)
+    L1 = rng.standard_normal((rank, K)).astype(np.float32) if rank else None
+    L2 = (rng.standard_normal((N, rank)) * 0.1).astype(np.float32) if rank else None
+    gx = 2.0 ** int(rng.integers(-8, 3)) if fmt == "nvfp4" else 1.0
+    _check_pack(fmt, R, L1, L2, gx)
