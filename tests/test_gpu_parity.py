@@ -319,3 +319,31 @@ def test_prologue_codes_exhaustive_over_bf16(fmt, gmax):
     X = I.to_bf16(allg.reshape(rows, K))
     assert np.array_equal(X, allg.reshape(rows, K))           # every value is already bf16
     _check_prologue(fmt, X, None, 1.0, None)
+
+
+@pytest.mark.parametrize("case", range(16))
+def test_layer_random_shapes(case):
+    """Seeded random shapes (ragged M, any multiple of 128 for N and K, every rank step) in
+    every format, through both calls; the same bars as the fixed cases."""
+    rng = np.random.default_rng(9000 + case)
+    fmt = ["nvfp4", "int4", "mxfp4", "w8a8"][case % 4]
+    M = int(rng.integers(1, 700))
+    N = 128 * int(rng.integers(1, 9))
+    K = 128 * int(rng.integers(1, 11))
+    rank = 16 * int(rng.integers(0, 9))
+    layer, prep = _layer(M, K, N, rank, seed=9100 + case, fmt=fmt, outliers=min(4, K // 64))
+    gx = prep["act_gscale"]
+    pk = B.pack_weight_np(fmt, prep["R_nk"].astype(np.float32), prep["L1_rk"].astype(np.float32) if rank else None,
+                          prep["L2_nr"].astype(np.float32) if rank else None, gx)
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
+    got, ref = _check_prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"] if rank else None)
+    L2s_dev = torch.from_numpy(pk["L2_bf16"].view(np.int16)).cuda().view(torch.bfloat16) if rank else None
+    Y = run_gemm(fmt, M, N, K, rank, got["dev"]["codes"], got["dev"]["scales"], gx,
+                 pk["w_codes"], pk["w_scales"], pk["w_gscale"], got["dev"]["Z"], L2s_dev, layer.bias)
+    Yg = host_bf16(Y)
+    out = O.gemm_forward(ref["q"], gx, packed["q"], packed["gscale"], got["Z"] if rank else None,
+                         packed["L2_bf16"] if rank else None, layer.bias)
+    assert rel_fro(Yg, out["Y"]) <= Y_TOL
+    assert_y_elementwise(Yg, out["Y64"], y_elementwise_slack(ref["q"], gx, packed["q"], packed["gscale"],
+                                                             got["Z"] if rank else None,
+                                                             packed["L2_bf16"] if rank else None, layer.bias))
