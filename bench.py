@@ -544,6 +544,39 @@ def main():
         gemm0.append((a, b))
     torch.cuda.synchronize()
     t_gemm0 = sum(a.elapsed_time(b) for a, b in gemm0) / len(gemm0) * 1e-3
+    # Library reference for the plain 4-bit product (no branch, no bias): cuBLASLt's NVFP4
+    # GEMM through torch._scaled_mm on the very same code and scale buffers (the 128x4
+    # blocked scale layout is the one cuBLASLt takes).  Context only, not part of any value.
+    library = None
+    if fmt == "nvfp4" and hasattr(torch, "float4_e2m1fn_x2"):
+        try:
+            ws = lin.workspace(M)
+            A4 = ws["a_codes"].view(torch.float4_e2m1fn_x2).view(M, K // 2)
+            W4 = lin.w_codes.view(torch.float4_e2m1fn_x2).view(N, K // 2).t()
+            sa = ws["a_scales"].view(torch.float8_e4m3fn)
+            sb = lin.w_scales.view(torch.float8_e4m3fn)
+            lin.prologue_only(X)
+            lin.gemm_only(M, Y, rank=0)
+            Yl = torch._scaled_mm(A4, W4, sa, sb, out_dtype=torch.bfloat16)
+            Yours = Y.float() - (lin.bias.float() if lin.bias is not None else 0.0)
+            rel = float((Yl.float() * (lin.act_gscale * lin.w_gscale) - Yours).norm() / Yours.norm())
+            lt = []
+            for i in range(args.warmup + max(5, args.steps // 2)):
+                flush.zero_()
+                a = torch.cuda.Event(enable_timing=True)
+                b = torch.cuda.Event(enable_timing=True)
+                a.record(stream)
+                torch._scaled_mm(A4, W4, sa, sb, out_dtype=torch.bfloat16)
+                b.record(stream)
+                if i >= args.warmup:
+                    lt.append((a, b))
+            torch.cuda.synchronize()
+            t_lib = sum(a.elapsed_time(b) for a, b in lt) / len(lt) * 1e-3
+            library = {"kernel": "cuBLASLt NVFP4 GEMM (torch._scaled_mm), same operands, rank 0, no bias",
+                       "us": t_lib * 1e6, "tflops": 2.0 * M * N * K / t_lib / 1e12,
+                       "ours_rank0_us": t_gemm0 * 1e6, "rel_fro_vs_ours": rel}
+        except Exception as e:                          # a torch build without the FP4 path
+            library = {"unavailable": f"{type(e).__name__}: {str(e)[:120]}"}
     # Fusion: the layer without the branch (prologue and GEMM at rank 0), and the same layer
     # with an unfused branch as separate passes (msModelSlim's two-path forward: the residual
     # linear's output plus two chained low-rank linears): X / lambda -> bf16, Z = X_hat L1^T,
@@ -698,6 +731,7 @@ def main():
             "unfused_vs_fused_rel_fro": fusion["rel"]},
         "gpu_launches": launches,
         "clocks": clk,
+        "library_reference": library,
         "step_us": step_dist,
         "hot_l2_ms_per_step": t_hot * 1e3,
     }
