@@ -401,3 +401,21 @@ def test_int8_rowwise_dequant_is_per_row_scale_times_code():
         for k in (0, 17, 255):
             assert deq[i, k] == float(q["scale"][i, 0]) * int(np.int8(q["codes"][i, k]))
     assert np.all(np.abs(x - deq) <= q["scale"].astype(np.float64) * (0.5 + 2.0 ** -16))
+
+
+def test_planted_w8a8_mistakes_are_caught(monkeypatch):
+    """A 128 code range (instead of 127) or scales taken per column (a transposed operand)
+    must break the eq.(1) worked example the W8A8 pins rest on."""
+    x = np.zeros((2, 128), np.float32)
+    x[0, 0] = 127.0
+    x[0, 1:4] = [2.5, 3.5, -126.5]
+    x[1, 0] = -1.0
+    good = O.quantize_int8_rowwise(x)
+    assert good["scale"][0, 0] == 1.0 and list(good["q"][0, :4]) == [127, 2, 4, -126]
+    import oracle.svdq_oracle as OM
+    monkeypatch.setattr(OM, "INT8_QMAX", 128)
+    wide = O.quantize_int8_rowwise(x)
+    assert wide["scale"][0, 0] != 1.0
+    monkeypatch.undo()
+    per_col = O.quantize_int8_rowwise(np.ascontiguousarray(x.T))
+    assert per_col["scale"].shape[0] != good["scale"].shape[0] or per_col["scale"][0, 0] != 1.0

@@ -221,3 +221,19 @@ def test_torch_prepare_one_iteration_unchanged(tiny):
     # the iterated split packs to a layer with a smaller calibration output error
     errs = b["residual"]["errors"]
     assert errs[b["residual"]["chosen"]] < errs[0]
+
+
+def test_planted_dropped_quantizer_is_caught(tiny):
+    """An iteration that refits to W_tilde - R_prev (Q dropped) returns the previous branch;
+    the refit pin (strictly better than the stale branch) catches it."""
+    _, _, Wt, _ = tiny
+    fmt, r = "nvfp4", 16
+    prev = O.residual_iteration(fmt, Wt, r, 1)
+    # the planted mistake, written out: refit to W_tilde - R instead of W_tilde - Q(R)
+    wrong = O.svd_split(Wt - prev["R"].astype(np.float64), r)
+    T = Wt - _deployed_qdq(fmt, prev["R"].astype(np.float64))
+    fit_wrong = np.linalg.norm(T - wrong["L1_bf16"] @ wrong["L2_bf16"])
+    stale = np.linalg.norm(T - prev["L1_bf16"] @ prev["L2_bf16"])
+    assert not fit_wrong < stale * (1 - 1e-3)          # the pin would fail on it
+    cur = O.residual_iteration(fmt, Wt, r, 2)
+    assert np.linalg.norm(T - cur["L1_bf16"] @ cur["L2_bf16"]) < stale
