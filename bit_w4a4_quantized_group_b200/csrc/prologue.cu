@@ -16,6 +16,11 @@
 // shared memory and written back as 16-byte row segments.  Z partials of the
 // warps that share a row strip are summed in a fixed order (deterministic).
 //
+// Few rows (small batches) leave most SMs idle, since a CTA owns 32 rows over all of K.  The
+// 4-bit formats then split each row block's K stages over a cluster of up to 4 CTAs: codes
+// and scales are local to their groups, and the Z partials of the CTAs are added by CTA 0
+// of the cluster through distributed shared memory, in CTA order (deterministic).
+//
 // W8A8 (the 8-bit setting: one scale per token row over all of K) needs each row's
 // maximum before any code can be formed, so the kernel makes two passes over its rows:
 // the first forms X_hat, the Z products and the row maxima; the compute warps then
@@ -141,11 +146,16 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int m0 = blockIdx.x * kProRows;
-  const int nkt = (p.K + BK - 1) / BK;
-  // Every CTA reads all of L1; starting the K loop at a different stage per CTA spreads
-  // those reads over the L2 instead of sending every SM to the same lines at once.
-  const int kt0 = blockIdx.x % nkt;
+  const int split = static_cast<int>(blockIdx.x) % p.ksplit;     // rank in the K-split cluster
+  const int rb = static_cast<int>(blockIdx.x) / p.ksplit;        // row block
+  const int m0 = rb * kProRows;
+  const int nkt_all = (p.K + BK - 1) / BK;
+  const int nks = (nkt_all + p.ksplit - 1) / p.ksplit;
+  const int kbeg = split * nks;                                   // this CTA's stages [kbeg, kbeg + nkt)
+  const int nkt = max(0, min(nkt_all, kbeg + nks) - kbeg);
+  // Every CTA reads all of its L1 columns; starting the K loop at a different stage per CTA
+  // spreads those reads over the L2 instead of sending every SM to the same lines at once.
+  const int kt0 = nkt > 0 ? rb % nkt : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
@@ -173,7 +183,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
         lv[i] = (p.lam != nullptr && c < p.K) ? __ldg(p.lam + c) : 1.f;
       }
     };
-    load_lambda(kt0 % nkt);
+    if (nkt > 0) load_lambda(kbeg + kt0 % nkt);
     const int nit = NPASS * nkt;
     for (int it = 0; it < nit; ++it) {
       const int s = it % S;
@@ -181,7 +191,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       if (!wait_bounded(&empty[s], ph ^ 1u, abort_flag, p.err, kErrSiteProEmpty)) break;
       const int ki = it % nkt;
       const bool with_l1 = RANK > 0 && it < nkt;      // L1 is only needed by the first pass
-      const int kt = (kt0 + ki) % nkt;
+      const int kt = kbeg + (kt0 + ki) % nkt;
       const int col0 = kt * BK;
       const int nbox = min(BK, p.K - col0) / 64;
       uint8_t* st = smem + s * L.stage_bytes;
@@ -199,7 +209,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       float cur[BK / 32];
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) cur[i] = lv[i];
-      if (it + 1 < nit) load_lambda((kt0 + (it + 1) % nkt) % nkt);
+      if (it + 1 < nit) load_lambda(kbeg + (kt0 + (it + 1) % nkt) % nkt);
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) {
         lam_s[i * 32 + lane] = cur[i];
@@ -235,7 +245,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       const int s = it % S;
       const uint32_t ph = (it / S) & 1;
       if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
-      const int kt = (kt0 + ki) % nkt;
+      const int kt = kbeg + (kt0 + ki) % nkt;
       const int col0 = kt * BK + phase * 64;
       if (col0 < p.K) {
         const uint8_t* st = smem + s * L.stage_bytes;
@@ -542,13 +552,46 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
             s1 += src[1];
           }
           const int row = m0 + strip * 16 + r;
-          if (row < p.M) {
+          if (p.ksplit > 1) {
+            float* zsum = zbuf + BOXES * 2 * 16 * R1;         // this CTA's partial [32][RANK]
+            zsum[(strip * 16 + r) * R1 + c] = s0;
+            zsum[(strip * 16 + r) * R1 + c + 1] = s1;
+          } else if (row < p.M) {
             __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
             *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * R1 + c) = v;
           }
         }
       }
     }
+  }
+
+  // K split over a cluster: CTA 0 adds the other CTAs' Z partials (read through distributed
+  // shared memory, in CTA order) and writes Z.  Every thread of every CTA reaches both
+  // cluster barriers; a wait that ran out above only ends its loop early.
+  if (RANK > 0 && p.ksplit > 1) {
+    constexpr int R1 = RANK > 0 ? RANK : 1;
+    ptx::cluster_sync();                                      // every partial is in shared memory
+    if (split == 0 && warp < 2) {
+      const int strip = warp;                                 // warps 0 and 1: phase 0, both strips
+      const float* zsum = reinterpret_cast<const float*>(smem) + BOXES * 2 * 16 * R1;
+      const uint32_t zaddr = ptx::smem_u32(zsum);
+      for (int idx = lane; idx < 16 * R1 / 2; idx += 32) {
+        const int r = (idx * 2) / R1, c = (idx * 2) % R1;
+        const int o = (strip * 16 + r) * R1 + c;
+        float s0 = zsum[o], s1 = zsum[o + 1];
+        for (int q = 1; q < p.ksplit; ++q) {
+          const uint32_t a = ptx::mapa_shared(zaddr + static_cast<uint32_t>(o) * 4u, static_cast<uint32_t>(q));
+          s0 += ptx::ld_shared_cluster_f32(a);
+          s1 += ptx::ld_shared_cluster_f32(a + 4u);
+        }
+        const int row = m0 + strip * 16 + r;
+        if (row < p.M) {
+          __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
+          *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * R1 + c) = v;
+        }
+      }
+    }
+    ptx::cluster_sync();                                      // peers keep their partials until read
   }
 }
 
@@ -578,8 +621,42 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
   auto kern = prologue_kernel<FMT, RANK>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
   if (e != cudaSuccess) return e;
-  const int grid = p.Mpad / kProRows;
-  kern<<<grid, 32 * (compute_warps(RANK) + 1), smem, stream>>>(tx, tl1, p);
+  const int blocks = p.Mpad / kProRows;
+  // K split for small batches (4-bit formats): the largest cluster of up to 4 CTAs per row
+  // block that keeps one wave on the SMs and leaves no CTA without a stage.
+  constexpr int BK = 64 * (compute_warps(RANK) / 2);
+  const int nkt_all = (p.K + BK - 1) / BK;
+  int sms = 0, dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    return cudaErrorInvalidDevice;
+  p.ksplit = 1;
+  if (FMT != kFmtW8a8 && RANK > 0) {
+    for (int ks = 4; ks >= 2; --ks) {
+      const int nks = (nkt_all + ks - 1) / ks;
+      if (ks <= nkt_all && nks * (ks - 1) < nkt_all && blocks * ks <= sms) {
+        p.ksplit = ks;
+        break;
+      }
+    }
+  }
+  if (p.ksplit == 1) {
+    kern<<<blocks, 32 * (compute_warps(RANK) + 1), smem, stream>>>(tx, tl1, p);
+    return cudaGetLastError();
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks * p.ksplit, 1, 1);
+  cfg.blockDim = dim3(32 * (compute_warps(RANK) + 1), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(p.ksplit);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, kern, tx, tl1, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

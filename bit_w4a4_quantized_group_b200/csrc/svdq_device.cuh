@@ -83,6 +83,7 @@ cudaError_t launch_selftest_bounded_wait(int* err, uint64_t limit_ns, cudaStream
 
 struct ProParams {
   int M, K, rank, Mpad, stages;
+  int ksplit;                // CTAs of a cluster that split one row block's K stages (1: none)
   const float* lam;          // nullable
   float gscale;              // activation tensor scale (NVFP4), 1 for INT4
   uint8_t* codes;            // [M][K/2] (W8A8: [M][K])

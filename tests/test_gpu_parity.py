@@ -63,7 +63,7 @@ def _check_prologue(fmt, X, lam, gx, L1_rk):
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
-                                      (96, 512, 128)])
+                                      (96, 512, 128), (256, 3072, 32), (100, 2048, 16), (64, 1280, 128)])
 def test_prologue_parity(fmt, M, K, rank):
     layer, prep = _layer(M, K, 256, rank, seed=7 + M + rank, fmt=fmt)
     _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
@@ -347,3 +347,22 @@ def test_layer_random_shapes(case):
     assert_y_elementwise(Yg, out["Y64"], y_elementwise_slack(ref["q"], gx, packed["q"], packed["gscale"],
                                                              got["Z"] if rank else None,
                                                              packed["L2_bf16"] if rank else None, layer.bias))
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("M,K,N,rank", [(256, 3072, 3072, 32), (1024, 3072, 1024, 64), (40, 2048, 512, 16)])
+def test_layer_small_batch_k_split(fmt, M, K, N, rank):
+    """Small batches, where the prologue splits each row block's K stages over a cluster of
+    CTAs and adds their Z partials through distributed shared memory; the whole layer
+    against the reference."""
+    layer, prep = _layer(M, K, N, rank, seed=77 + M + rank, fmt=fmt)
+    gx = prep["act_gscale"]
+    pk = B.pack_weight_np(fmt, prep["R_nk"].astype(np.float32), prep["L1_rk"].astype(np.float32),
+                          prep["L2_nr"].astype(np.float32), gx)
+    packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
+    got, ref = _check_prologue(fmt, layer.X, prep["lam"], gx, packed["L1_bf16"])
+    L2s_dev = torch.from_numpy(pk["L2_bf16"].view(np.int16)).cuda().view(torch.bfloat16)
+    Y = run_gemm(fmt, M, N, K, rank, got["dev"]["codes"], got["dev"]["scales"], gx,
+                 pk["w_codes"], pk["w_scales"], pk["w_gscale"], got["dev"]["Z"], L2s_dev, layer.bias)
+    out = O.gemm_forward(ref["q"], gx, packed["q"], packed["gscale"], got["Z"], packed["L2_bf16"], layer.bias)
+    assert rel_fro(host_bf16(Y), out["Y"]) <= Y_TOL
