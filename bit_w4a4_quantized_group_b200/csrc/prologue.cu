@@ -123,7 +123,7 @@ __device__ __forceinline__ float div_code(float a, float b, float y) {
 __host__ __device__ constexpr int code_stage_bytes(int fmt) { return fmt == kFmtW8a8 ? 1024 : 512; }
 __host__ __device__ constexpr int passes(int fmt) { return fmt == kFmtW8a8 ? 2 : 1; }
 
-template <int FMT, int RANK>
+template <int FMT, int RANK, bool SPLIT>
 __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     prologue_kernel(const __grid_constant__ CUtensorMap tmap_x, const __grid_constant__ CUtensorMap tmap_l1,
                     ProParams p) {
@@ -146,13 +146,13 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int split = static_cast<int>(blockIdx.x) % p.ksplit;     // rank in the K-split cluster
-  const int rb = static_cast<int>(blockIdx.x) / p.ksplit;        // row block
+  const int split = SPLIT ? static_cast<int>(blockIdx.x) % p.ksplit : 0;   // rank in the K-split cluster
+  const int rb = SPLIT ? static_cast<int>(blockIdx.x) / p.ksplit : static_cast<int>(blockIdx.x);  // row block
   const int m0 = rb * kProRows;
   const int nkt_all = (p.K + BK - 1) / BK;
-  const int nks = (nkt_all + p.ksplit - 1) / p.ksplit;
+  const int nks = SPLIT ? (nkt_all + p.ksplit - 1) / p.ksplit : nkt_all;
   const int kbeg = split * nks;                                   // this CTA's stages [kbeg, kbeg + nkt)
-  const int nkt = max(0, min(nkt_all, kbeg + nks) - kbeg);
+  const int nkt = SPLIT ? max(0, min(nkt_all, kbeg + nks) - kbeg) : nkt_all;
   // Every CTA reads all of its L1 columns; starting the K loop at a different stage per CTA
   // spreads those reads over the L2 instead of sending every SM to the same lines at once.
   const int kt0 = nkt > 0 ? rb % nkt : 0;
@@ -552,7 +552,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
             s1 += src[1];
           }
           const int row = m0 + strip * 16 + r;
-          if (p.ksplit > 1) {
+          if (SPLIT) {
             float* zsum = zbuf + BOXES * 2 * 16 * R1;         // this CTA's partial [32][RANK]
             zsum[(strip * 16 + r) * R1 + c] = s0;
             zsum[(strip * 16 + r) * R1 + c + 1] = s1;
@@ -568,7 +568,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   // K split over a cluster: CTA 0 adds the other CTAs' Z partials (read through distributed
   // shared memory, in CTA order) and writes Z.  Every thread of every CTA reaches both
   // cluster barriers; a wait that ran out above only ends its loop early.
-  if (RANK > 0 && p.ksplit > 1) {
+  if (RANK > 0 && SPLIT) {
     constexpr int R1 = RANK > 0 ? RANK : 1;
     ptx::cluster_sync();                                      // every partial is in shared memory
     if (split == 0 && warp < 2) {
@@ -618,9 +618,6 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
   p.stages = stages_for<FMT, RANK>();
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = smem_bytes_for<FMT, RANK>(p.stages);
-  auto kern = prologue_kernel<FMT, RANK>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-  if (e != cudaSuccess) return e;
   const int blocks = p.Mpad / kProRows;
   // K split for small batches (4-bit formats): the largest cluster of up to 4 CTAs per row
   // block that keeps one wave on the SMs and leaves no CTA without a stage.
@@ -640,9 +637,15 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
     }
   }
   if (p.ksplit == 1) {
+    auto kern = prologue_kernel<FMT, RANK, false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
     kern<<<blocks, 32 * (compute_warps(RANK) + 1), smem, stream>>>(tx, tl1, p);
     return cudaGetLastError();
   }
+  auto kern = prologue_kernel<FMT, RANK, true>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks * p.ksplit, 1, 1);
   cfg.blockDim = dim3(32 * (compute_warps(RANK) + 1), 1, 1);
