@@ -627,7 +627,7 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return cudaErrorInvalidDevice;
   p.ksplit = 1;
-  if (FMT != kFmtW8a8 && RANK > 0) {
+  if (FMT != kFmtW8a8) {
     for (int ks = 4; ks >= 2; --ks) {
       const int nks = (nkt_all + ks - 1) / ks;
       if (ks <= nkt_all && nks * (ks - 1) < nkt_all && blocks * ks <= sms) {

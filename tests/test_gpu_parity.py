@@ -63,7 +63,8 @@ def _check_prologue(fmt, X, lam, gx, L1_rk):
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
-                                      (96, 512, 128), (256, 3072, 32), (100, 2048, 16), (64, 1280, 128)])
+                                      (96, 512, 128), (256, 3072, 32), (100, 2048, 16), (64, 1280, 128),
+                                      (64, 2048, 0), (200, 3072, 0)])
 def test_prologue_parity(fmt, M, K, rank):
     layer, prep = _layer(M, K, 256, rank, seed=7 + M + rank, fmt=fmt)
     _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
