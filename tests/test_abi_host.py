@@ -237,3 +237,14 @@ def test_pack_weight_matches_reference_randomized(lib, fmt, nb, kb, rank, exp, d
     L2 = (rng.standard_normal((N, rank)) * 0.1).astype(np.float32) if rank else None
     gx = 2.0 ** int(rng.integers(-8, 3)) if fmt == "nvfp4" else 1.0
     _check_pack(fmt, R, L1, L2, gx)
+
+
+def test_missing_library_fails_loudly(tmp_path, monkeypatch):
+    """No CPU fallback: without the built library the binding raises instead of computing."""
+    monkeypatch.setattr(B, "_lib", None)
+    with pytest.raises(RuntimeError, match="libsvdq.so not found"):
+        B.load(str(tmp_path / "libsvdq.so"))
+    import oracle  # noqa: F401  (the reference is importable, but the product path never uses it)
+    import bit_w4a4_quantized_group_b200.layer as L
+    src = open(L.__file__, encoding="utf-8").read() + open(B.__file__, encoding="utf-8").read()
+    assert "oracle" not in src
