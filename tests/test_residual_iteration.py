@@ -237,3 +237,32 @@ def test_planted_dropped_quantizer_is_caught(tiny):
     assert not fit_wrong < stale * (1 - 1e-3)          # the pin would fail on it
     cur = O.residual_iteration(fmt, Wt, r, 2)
     assert np.linalg.norm(T - cur["L1_bf16"] @ cur["L2_bf16"]) < stale
+
+
+def test_offline_tensor_scale_matches_the_reference():
+    """prepare.py's power-of-two tensor scale (reading 4) against the reference's, at the
+    exact boundaries 6 * 448 * 2^e, one ulp either side of them, zero and random values."""
+    rng = np.random.default_rng(55)
+    vals = [0.0, 1e-30, 3.0e38]
+    for e in range(-40, 40, 3):
+        b = 6.0 * 448.0 * 2.0 ** e
+        vals += [b, float(np.nextafter(np.float32(b), np.float32(np.inf))),
+                 float(np.nextafter(np.float32(b), np.float32(0)))]
+    vals += list(np.exp(rng.uniform(-60, 60, 200)))
+    for v in vals:
+        v32 = float(np.float32(v))
+        assert P.pow2_tensor_scale(v32) == O.pow2_global_scale(v32), v32
+
+
+def test_offline_prepare_matches_the_reference_split(tiny):
+    """prepare.py (PyTorch, fp64 SVD) against the reference's prepare_layer on the same layer:
+    lambda and g_x bit for bit, the bf16 factors' product and the residual to SVD rounding."""
+    layer = tiny[0]
+    for fmt in FMTS:
+        a = P.prepare(fmt, layer.X, layer.W, 16, device="cpu")
+        ref = O.prepare_layer(fmt, layer.X, layer.W, 16)
+        assert np.array_equal(a["lam"], ref["lam"]) and a["act_gscale"] == ref["act_gscale"]
+        prod = a["L2_nr"].astype(np.float64) @ a["L1_rk"].astype(np.float64)
+        prod_ref = ref["L2_nr"] @ ref["L1_rk"]
+        assert np.linalg.norm(prod - prod_ref) <= 1e-2 * np.linalg.norm(prod_ref)
+        assert np.linalg.norm(a["R_nk"] - ref["R_nk"]) <= 2e-2 * np.linalg.norm(ref["R_nk"]) + 1e-6
