@@ -32,11 +32,21 @@ class W4A4LowRankLinear:
         self.act_gscale = float(act_gscale)
         self.L1 = _to_dev_u16_as_bf16(packed["L1_bf16"], self.device) if self.rank else None
         self.L2 = _to_dev_u16_as_bf16(packed["L2_bf16"], self.device) if self.rank else None
-        self.lam = None if lam is None else torch.from_numpy(np.ascontiguousarray(lam, np.float32)).to(self.device)
+        if lam is not None:
+            lam32 = np.ascontiguousarray(lam, np.float32)
+            # the smoothing divide x / lambda is an IEEE divide only for finite, normal, positive
+            # lambda (the C ABI's contract); anything else is rejected here, before any launch
+            tiny = np.finfo(np.float32).tiny
+            if lam32.shape != (self.K,) or not np.all(np.isfinite(lam32) & (lam32 >= tiny)):
+                raise ValueError("lambda must hold K finite, normal, positive float32 values")
+            self.lam = torch.from_numpy(lam32).to(self.device)
+        else:
+            self.lam = None
         self.bias = None
         if bias is not None:
-            bits = (np.ascontiguousarray(bias, np.float32).view(np.uint32) >> 16).astype(np.uint16)
-            self.bias = _to_dev_u16_as_bf16(bits, self.device)
+            # bf16 by round-to-nearest-even (torch's conversion), like every other bf16 operand
+            b32 = torch.from_numpy(np.ascontiguousarray(bias, np.float32).reshape(-1))
+            self.bias = b32.to(torch.bfloat16).to(self.device)
         self._ws = {}
 
     def workspace(self, M: int):
@@ -50,7 +60,15 @@ class W4A4LowRankLinear:
             }
         return self._ws[M]
 
-    def forward(self, X: torch.Tensor, Y: Optional[torch.Tensor] = None) -> torch.Tensor:
+    def forward(self, X: torch.Tensor, Y: Optional[torch.Tensor] = None, check: bool = False) -> torch.Tensor:
+        """Y = the layer applied to X (both calls on the current stream, asynchronous).
+
+        With ``check=True`` the call also synchronizes the stream and reads the library's
+        device error word: a kernel whose bounded wait ran out (for instance on a GPU that
+        is time-sliced with other work) leaves Y undefined, and this raises instead of
+        returning it.  Without it, callers that need the guarantee poll
+        ``binding.svdq_get_last_device_error`` themselves.
+        """
         M, K = X.shape
         ws = self.workspace(M)
         if Y is None:
@@ -60,6 +78,10 @@ class W4A4LowRankLinear:
         B.w4a4_gemm_lowrank_up_t(self.fmt, M, self.N, K, self.rank, ws["a_codes"], ws["a_scales"],
                                  self.act_gscale, self.w_codes, self.w_scales, self.w_gscale,
                                  ws["Z"], self.L2, self.bias, Y)
+        if check:
+            st, site = B.svdq_get_last_device_error(torch.cuda.current_stream(self.device).cuda_stream)
+            if st != B.SVDQ_OK:
+                raise B.SvdqError(st, f"layer forward (device wait site {site})")
         return Y
 
     def gemm_only(self, M: int, Y: torch.Tensor, rank: Optional[int] = None):
