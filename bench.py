@@ -342,6 +342,25 @@ def whole_job_tflops(world, flops_per_rank, seconds):
     return world * flops_per_rank / seconds / 1e12
 
 
+def layer_algorithmic(fmt, M, K, N, r):
+    """Algorithmic bytes of the prologue and of the GEMM, and the GEMM's FLOPs (2MNK + 2MNr).
+
+    Prologue: X (2MK), codes and scales, Z (2Mr), L1 (2rK) and lambda (4K).  GEMM: both
+    operands' codes and scales, Z, L2 (2Nr), bias (2N) and Y (2MN).  Codes are half a byte
+    per element (W8A8: one); scales one byte per 16 (NVFP4) or 32 (MXFP4) elements, two per
+    64 (INT4 fp16), four per row (W8A8 fp32).
+    """
+    if fmt == "w8a8":
+        code, sc = 1.0, lambda rows: 4.0 * rows
+    else:
+        g = {"nvfp4": 16, "mxfp4": 32, "int4": 64}[fmt]
+        per = 2.0 if fmt == "int4" else 1.0
+        code, sc = 0.5, (lambda rows: rows * K / g * per)
+    pro = 2.0 * M * K + code * M * K + sc(M) + 2.0 * M * r + 2.0 * r * K + 4.0 * K
+    gemm = code * (M + N) * K + sc(M) + sc(N) + 2.0 * M * r + 2.0 * N * r + 2.0 * N + 2.0 * M * N
+    return pro, gemm, 2.0 * M * N * K + 2.0 * M * N * r
+
+
 def config_dict(cfg, fmt, l2):
     return {"workload": f"{cfg.name} {cfg.b}x{cfg.m}x{cfg.n} r={cfg.rank} {fmt}", "M": cfg.b, "K": cfg.m,
             "N": cfg.n, "rank": cfg.rank, "format": fmt, "bias": cfg.with_bias, "l2": l2}
@@ -373,7 +392,7 @@ def run_sweep(args):
     fmt = args.format
     stream = torch.cuda.current_stream()
     flush = torch.empty(512 * 1024 * 1024, dtype=torch.uint8, device=device)
-    bf16_burst, _, _, _ = peaks()
+    bf16_burst, _, hbm, peak_src = peaks()
     peak = bf16_burst * (4.0 if fmt in ("nvfp4", "mxfp4") else 2.0)
 
     def timed(fn, n):
@@ -411,11 +430,23 @@ def run_sweep(args):
         t_pro = timed(lambda: lin.prologue_only(X), n)
         t_gemm = timed(lambda: lin.gemm_only(M, Y), n)
         t_r0 = timed(lambda: (lin.prologue_only(X, rank=0), lin.gemm_only(M, Y, rank=0)), n)
+        pro_b, gemm_b, gemm_f = layer_algorithmic(fmt, M, K, N, r)
+        # the two kernels run one after the other: each is bound by its own roofline
+        t_pro_roof = pro_b / (hbm * 1e9)
+        t_gemm_hbm = gemm_b / (hbm * 1e9)
+        t_gemm_tc = gemm_f / (peak * 1e12)
+        t_roof = t_pro_roof + max(t_gemm_hbm, t_gemm_tc)
         out = {"sweep_point": cfg.name, "format": fmt, "M": M, "K": K, "N": N, "rank": r,
                "lora_rank": cfg.lora_rank, "layer_us": t_layer * 1e6, "prologue_us": t_pro * 1e6,
                "gemm_us": t_gemm * 1e6, "tflops": 2.0 * M * N * K / t_layer / 1e12,
                "gemm_frac": (2.0 * M * N * K + 2.0 * M * N * r) / t_gemm / 1e12 / peak,
-               "layer_r0_us": t_r0 * 1e6, "fused_overhead_pct": 100.0 * (t_layer / t_r0 - 1.0)}
+               "layer_r0_us": t_r0 * 1e6, "fused_overhead_pct": 100.0 * (t_layer / t_r0 - 1.0),
+               "roofline": {"gemm_bound": "hbm" if t_gemm_hbm > t_gemm_tc else "tensor",
+                            "layer_roof_us": t_roof * 1e6, "frac": t_roof / t_layer,
+                            "gemm_roof_us": max(t_gemm_hbm, t_gemm_tc) * 1e6,
+                            "gemm_frac": max(t_gemm_hbm, t_gemm_tc) / t_gemm,
+                            "prologue_roof_us": t_pro_roof * 1e6, "prologue_frac": t_pro_roof / t_pro,
+                            "peaks": f"{peak_src}: HBM {hbm:.0f} GB/s, tensor {peak:.0f} TFLOP/s"}}
         if r > 0:
             up_scale = lin.act_gscale * lin.w_gscale
             lam_d = torch.ones(K, device=device)
