@@ -11,27 +11,33 @@
 // B200 design (one CTA per SM, 128 x 128 output tiles, persistent):
 //   * a producer warp streams the packed codes of 128-column K steps into a
 //     3-deep ring with TMA (64B-swizzled, so the row reads below are free of
-//     bank conflicts); four widening warps turn every code q into the int8 byte
+//     bank conflicts); two widening warps turn every code q into the int8 byte
 //     16 q in the 128B-swizzled K-major layout of the MMA, in a second 3-deep
-//     ring.  A nibble moved to the top of its byte *is* 16 q in two's complement,
+//     ring (two rows per thread).  A nibble moved to the top of its byte *is* 16 q in two's complement,
 //     so eight codes take two logic operations: the even nibbles of a 32-bit word
 //     go to one word, the odd ones to the next.  That permutes K inside every
 //     8-element chunk, identically for A and B, which leaves each group's dot
 //     product unchanged;
 //   * the MMA warp issues tcgen05 kind::i8 MMAs (s8 x s8 -> s32) per 64-element
 //     group into one of four TMEM group buffers.  Each buffer is preset to the
-//     bit pattern of the float 1.5 * 2^23, so after the MMAs it holds the fp32
-//     number 1.5 * 2^23 + 256 D_g exactly (|256 D_g| <= 2^20): subtracting
-//     1.5 * 2^23 recovers 256 D_g exactly without an int-to-float conversion;
-//   * eight epilogue warps drain each group buffer, preset it again, release it,
-//     and add 256 D_g * (s_x s_w / 256) in fp32 into register accumulators with
-//     packed f32x2 operations (the products and sums are those of D_g * s_x s_w);
-//     the low-rank branch is one more "group" (bf16 kind::f16 MMAs, scale 1)
+//     bit pattern of the float B = 1.5 * 2^23, so after the MMAs it holds the fp32
+//     number v = B + 256 D_g exactly (|256 D_g| <= 2^20);
+//   * eight epilogue warps (two per TMEM lane quarter, 64 columns each) drain
+//     each group buffer with two 32-column loads, preset it again while they
+//     scale the values, and hand it back; the group's scales are prepared before
+//     its product is waited for.
+//     The scaling takes two fp32 FMAs per element and group:
+//        t = fma(v, s_w/256, -B s_w/256) = RN(D_g s_w)  (B s_w/256 is exact, and
+//            the fma rounds v s_w/256 - B s_w/256 = D_g s_w once),
+//        acc = fma(t, s_x, acc),
+//     packed two columns at a time (f32x2); the per-column pairs (s_w/256,
+//     -B s_w/256) come from shared memory as one 16-byte broadcast per two columns;
+//   * the low-rank branch is one more "group" (bf16 kind::f16 MMAs, added as is)
 //     whose Z and L2 tiles the producer loads with TMA into their own slot;
-//   * Y leaves through 128B-swizzled shared-memory boxes and TMA stores.
-// The per-group fp32 scaling is CUDA-core work of the same order as the MMAs;
-// it is what the INT4 format costs next to NVFP4, whose group scales the
-// tensor cores apply themselves.
+//   * Y leaves through 128B-swizzled 32 x 64 shared-memory boxes and TMA stores.
+// The per-group fp32 scaling is CUDA-core work larger than the MMAs (two FMAs per
+// output element and group against the tensor core's 64 multiply-adds); it is what
+// the INT4 format costs next to NVFP4, whose group scales the tensor cores apply.
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
@@ -45,10 +51,12 @@ namespace {
 
 constexpr int kBM = 128, kBN = 128;
 constexpr int kKStep = 128;                    // elements per pipeline step (two groups)
-constexpr int kStages = 3;                     // widened (E4M3) ring
+constexpr int kStages = 3;                     // widened (int8) ring
 constexpr int kPkStages = 3;                   // packed-code ring
-constexpr int kLoadWarps = 4, kMmaWarp = 4, kProdWarp = 5, kEpiWarp0 = 6, kEpiWarps = 8;
-constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);   // 448
+// 12 warps (three per SM sub-partition, whose 16K registers then allow 168 per thread):
+// two widening warps (two tile rows per thread), the MMA warp, the producer, 8 epilogue warps
+constexpr int kLoadWarps = 2, kMmaWarp = 2, kProdWarp = 3, kEpiWarp0 = 4, kEpiWarps = 8;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);   // 384
 constexpr uint32_t kOpBytes = kBM * 128;       // 16 KB: 128 rows x 128 bytes
 constexpr uint32_t kStageBytes = 2 * kOpBytes; // A then B
 constexpr uint32_t kPkOpBytes = kBM * 64;      // 8 KB: 128 rows x 64 packed bytes
@@ -57,6 +65,7 @@ constexpr uint32_t kLrBytes = 2 * kOpBytes;    // Z tile + L2 tile (bf16, 64 col
 constexpr int kScStages = 8;                   // group-scale ring, one slot per K step
 constexpr uint32_t kScBytes = 1024;            // s_x: 2 groups x 128 rows, s_w: 2 groups x 128 columns (fp16)
 constexpr uint32_t kEpiBoxBytes = 32 * 128;    // 32 rows x 64 bf16
+constexpr uint32_t kPairBytes = 2 * 128 * 4;   // per epilogue warp: two groups x 32 column pairs x 4 floats
 constexpr int kGroupBufs = 4;                  // TMEM: 4 x 128 fp32 columns
 
 __host__ __device__ constexpr uint32_t idesc_s8(int m, int n) {
@@ -64,7 +73,8 @@ __host__ __device__ constexpr uint32_t idesc_s8(int m, int n) {
   return (2u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
 }
-constexpr uint32_t kAccBias = 0x4B400000u;    // bits of 1.5 * 2^23
+constexpr uint32_t kAccBias = 0x4B400000u;    // bits of B = 1.5 * 2^23
+constexpr float kAccBiasF = 12582912.0f;
 __host__ __device__ constexpr uint32_t idesc_bf16(int m, int n) {
   return (1u << 4) | (1u << 7) | (1u << 10) | (static_cast<uint32_t>(n >> 3) << 17) |
          (static_cast<uint32_t>(m >> 4) << 24);
@@ -85,11 +95,18 @@ struct SharedTail {
   int abort_flag;
 };
 
+constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kPkStages * kPkStageBytes + kLrBytes +
+                              kScStages * kScBytes + kEpiWarps * kEpiBoxBytes + kEpiWarps * kPairBytes +
+                              sizeof(SharedTail);
+static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
+
 // Eight 4-bit two's complement codes (low nibble first) -> eight int8 bytes 16 q:
 // .x = codes 0, 2, 4, 6 and .y = codes 1, 3, 5, 7 (the K permutation described above).
 __device__ __forceinline__ uint2 int4x8_to_s8x8_x16(uint32_t w) {
   return make_uint2((w << 4) & 0xF0F0F0F0u, w & 0xF0F0F0F0u);
 }
+
+__device__ __forceinline__ float2 u2f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
@@ -102,8 +119,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* lr_smem = pk_smem + kPkStages * kPkStageBytes;
   uint8_t* sc_smem = lr_smem + kLrBytes;
   uint8_t* epi_smem = sc_smem + kScStages * kScBytes;
-  float* sbuf = reinterpret_cast<float*>(epi_smem + kEpiWarps * kEpiBoxBytes);   // 8 warps x 64 scales
-  SharedTail* sh = reinterpret_cast<SharedTail*>(sbuf + kEpiWarps * 64);
+  float* pair_smem = reinterpret_cast<float*>(epi_smem + kEpiWarps * kEpiBoxBytes);
+  SharedTail* sh = reinterpret_cast<SharedTail*>(reinterpret_cast<uint8_t*>(pair_smem) + kEpiWarps * kPairBytes);
   volatile int* abort_flag = &sh->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -112,8 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int G = K / 64;
   const int nk_main = (K + kKStep - 1) / kKStep;
   const int nk_lr = (p.rank + 63) / 64;
-  const int nk = nk_main + nk_lr;
-  const int K2 = K / 2;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -145,16 +160,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
-  if (warp >= kEpiWarp0) {
-    // preset every group buffer (this warp's 32 lanes x 64 columns of each) to the bias pattern
-    const uint32_t base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + ((warp - kEpiWarp0) >> 2) * 64;
-#pragma unroll
-    for (int b = 0; b < kGroupBufs; ++b) {
-      ptx::tmem_st_32x32b_x32_same(base + b * kBN, kAccBias);
-      ptx::tmem_st_32x32b_x32_same(base + b * kBN + 32, kAccBias);
-    }
-    ptx::tmem_wait_st();
-  }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
@@ -203,7 +208,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp < kLoadWarps) {
     // ------------------------------------------------------------ widening warps
-    const int r = threadIdx.x;                  // tile row handled by this thread (A and B)
     int it = 0;
     bool ok = true;
     for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
@@ -214,39 +218,47 @@ __global__ void __launch_bounds__(kThreads, 1)
           ok = false;
           break;
         }
-        // this row's 64 packed bytes of A and of B (64B-swizzled rows)
-        const uint8_t* pa = pk_smem + ps * kPkStageBytes + r * 64;
-        const uint8_t* pb = pa + kPkOpBytes;
-        const int sw = (r >> 1) & 3;
-        uint4 va[4], vb[4];
+        // rows r and r + 64 of the tile (A and B): 64 packed bytes each, 64B-swizzled rows
+        uint4 va[2][4], vb[2][4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          va[i] = *reinterpret_cast<const uint4*>(pa + ((i ^ sw) << 4));
-          vb[i] = *reinterpret_cast<const uint4*>(pb + ((i ^ sw) << 4));
+        for (int h = 0; h < 2; ++h) {
+          const int r = threadIdx.x + 64 * h;
+          const uint8_t* pa = pk_smem + ps * kPkStageBytes + r * 64;
+          const uint8_t* pb = pa + kPkOpBytes;
+          const int sw = (r >> 1) & 3;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            va[h][i] = *reinterpret_cast<const uint4*>(pa + ((i ^ sw) << 4));
+            vb[h][i] = *reinterpret_cast<const uint4*>(pb + ((i ^ sw) << 4));
+          }
         }
         ptx::mbar_arrive(&sh->pk_empty[ps]);
         if (!wait_bounded(&sh->empty[s], ((it / kStages) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmConvEmpty)) {
           ok = false;
           break;
         }
-        uint8_t* arow_s = smem + s * kStageBytes + r * 128;
-        uint8_t* brow_s = arow_s + kOpBytes;
-        // 64 packed bytes -> 128 E4M3 bytes = 8 chunks of 16 bytes, 128B-swizzled by row
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint32_t wa[4] = {va[i].x, va[i].y, va[i].z, va[i].w};
-          const uint32_t wb[4] = {vb[i].x, vb[i].y, vb[i].z, vb[i].w};
-          uint2 ea[4], eb[4];
+        for (int h = 0; h < 2; ++h) {
+          const int r = threadIdx.x + 64 * h;
+          uint8_t* arow_s = smem + s * kStageBytes + r * 128;
+          uint8_t* brow_s = arow_s + kOpBytes;
+          // 64 packed bytes -> 128 int8 bytes = 8 chunks of 16 bytes, 128B-swizzled by row
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            ea[j] = int4x8_to_s8x8_x16(wa[j]);
-            eb[j] = int4x8_to_s8x8_x16(wb[j]);
+          for (int i = 0; i < 4; ++i) {
+            const uint32_t wa[4] = {va[h][i].x, va[h][i].y, va[h][i].z, va[h][i].w};
+            const uint32_t wb[4] = {vb[h][i].x, vb[h][i].y, vb[h][i].z, vb[h][i].w};
+            uint2 ea[4], eb[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              ea[j] = int4x8_to_s8x8_x16(wa[j]);
+              eb[j] = int4x8_to_s8x8_x16(wb[j]);
+            }
+            const int c0 = 2 * i, c1 = 2 * i + 1;
+            *reinterpret_cast<uint4*>(arow_s + ((c0 ^ (r & 7)) << 4)) = make_uint4(ea[0].x, ea[0].y, ea[1].x, ea[1].y);
+            *reinterpret_cast<uint4*>(arow_s + ((c1 ^ (r & 7)) << 4)) = make_uint4(ea[2].x, ea[2].y, ea[3].x, ea[3].y);
+            *reinterpret_cast<uint4*>(brow_s + ((c0 ^ (r & 7)) << 4)) = make_uint4(eb[0].x, eb[0].y, eb[1].x, eb[1].y);
+            *reinterpret_cast<uint4*>(brow_s + ((c1 ^ (r & 7)) << 4)) = make_uint4(eb[2].x, eb[2].y, eb[3].x, eb[3].y);
           }
-          const int c0 = 2 * i, c1 = 2 * i + 1;
-          *reinterpret_cast<uint4*>(arow_s + ((c0 ^ (r & 7)) << 4)) = make_uint4(ea[0].x, ea[0].y, ea[1].x, ea[1].y);
-          *reinterpret_cast<uint4*>(arow_s + ((c1 ^ (r & 7)) << 4)) = make_uint4(ea[2].x, ea[2].y, ea[3].x, ea[3].y);
-          *reinterpret_cast<uint4*>(brow_s + ((c0 ^ (r & 7)) << 4)) = make_uint4(eb[0].x, eb[0].y, eb[1].x, eb[1].y);
-          *reinterpret_cast<uint4*>(brow_s + ((c1 ^ (r & 7)) << 4)) = make_uint4(eb[2].x, eb[2].y, eb[3].x, eb[3].y);
         }
         ptx::fence_proxy_async_smem();        // generic-proxy writes -> visible to the tensor cores
         ptx::mbar_arrive(&sh->full[s]);
@@ -279,8 +291,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int kk = 0; kk < 2; ++kk) {
               const uint32_t off = j * 64 + kk * 32;
-              // accumulate onto the preset bias pattern (see the header)
-              ptx::umma_i8(d, ptx::sdesc_sw128(st + off), ptx::sdesc_sw128(st + kOpBytes + off), id8, 1u);
+              // the group's first MMA overwrites the buffer (s32 256 D_g)
+              ptx::umma_i8(d, ptx::sdesc_sw128(st + off), ptx::sdesc_sw128(st + kOpBytes + off), id8, kk ? 1u : 0u);
             }
             ptx::tc_commit(&sh->grp_full[b]);
           }
@@ -290,7 +302,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       if (!ok || nk_lr == 0) continue;
-      // low-rank branch: Z L2^T into one more group buffer
+      // low-rank branch: Z L2^T into one more group buffer (its first MMA overwrites the preset)
       const int b = gi % kGroupBufs;
       if (!wait_bounded(&sh->grp_empty[b], ((gi / kGroupBufs) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmAccEmpty)) {
         ok = false;
@@ -317,107 +329,109 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++gi;
     }
   } else {
-    // ------------------------------------------------------------ epilogue (warps 6-13)
+    // ------------------------------------------------------------ epilogue (warps 4-11)
+    // Each warp owns 32 rows (its TMEM lane quarter) x 64 columns and reads them in the
+    // 16x256b shape: thread l holds rows {l/4, l/4 + 8} of each 16-row slab and the column
+    // pairs 8i + 2(l%4) + {0, 1}, i = 0..7, i.e. 4 rows x 16 columns.  A thread then needs
+    // the weight-scale pairs of 16 columns per group (8 shared loads) instead of 64.
     const int e = warp - kEpiWarp0;
-    const int q = warp & 3;                    // TMEM lane quarter
+    const int q = warp & 3;                    // TMEM lane quarter (rows q*32 .. q*32+31)
     const int h = e >> 2;                      // 64-column half of the tile
-    float* sb_s = sbuf + e * 64;
+    const int lr = lane >> 2, lc = lane & 3;   // row within an 8-row group, column pair within a chunk
+    float* pairs = pair_smem + e * (kPairBytes / 4);
     uint8_t* buf = epi_smem + e * kEpiBoxBytes;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 64;
+    const int ngroups = G + (p.rank > 0 ? 1 : 0);
     int gi = 0, sc_it = 0;
-    for (int t = blockIdx.x; t < p.num_tiles; t += gridDim.x) {
+    bool ok = true;
+    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
       const int m0 = (t % p.tiles_m) * kBM, n0 = (t / p.tiles_m) * kBN;
       const int col0 = n0 + h * 64;
-      float2 acc[32];
+      float2 acc[4][8];                        // [row j = 2 slab + half][chunk i]
 #pragma unroll
-      for (int c = 0; c < 32; ++c) acc[c] = make_float2(0.f, 0.f);
-      bool ok = true;
-      const int ngroups = G + (p.rank > 0 ? 1 : 0);
+      for (int j = 0; j < 4; ++j)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[j][i] = make_float2(0.f, 0.f);
       for (int g = 0; g < ngroups; ++g, ++gi) {
         const bool lowrank = g == G;
-        float sa = 1.f;
-        const int kstep = g >> 1;
-        const int ss = (sc_it + kstep) % kScStages;
+        const int b = gi % kGroupBufs;
+        const uint32_t base = lane_base + b * kBN;
+        float sa[4] = {1.f, 1.f, 1.f, 1.f};
+        const float* pr = pairs + (g & 1) * 128;
         if (!lowrank) {
+          // this group's row scales and (s_w / 256, -B s_w / 256) for the warp's 64 columns
+          // (written by lane l for columns 2l, 2l + 1), prepared before the product is waited for
+          const int ss = (sc_it + (g >> 1)) % kScStages;
           if ((g & 1) == 0 &&
-              !wait_bounded(&sh->sc_full[ss], ((sc_it + kstep) / kScStages) & 1, abort_flag, p.err, kErrSiteGemmFull)) {
+              !wait_bounded(&sh->sc_full[ss], ((sc_it + (g >> 1)) / kScStages) & 1, abort_flag, p.err,
+                            kErrSiteGemmFull)) {
             ok = false;
             break;
           }
-          // this warp's 64 column scales of group g divided by 256 (exact), as fp32 in shared memory
           const uint8_t* sc = sc_smem + ss * kScBytes + (g & 1) * 256;
-          const float2 fb = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
-          sa = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + lane) * 2));
+#pragma unroll
+          for (int j = 0; j < 4; ++j)
+            sa[j] = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + 8 * j + lr) * 2));
+          const float2 sw = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
+          const float w0 = sw.x * 0.00390625f, w1 = sw.y * 0.00390625f;
+          *reinterpret_cast<float4*>(pairs + (g & 1) * 128 + lane * 4) =
+              make_float4(w0, w1, w0 * -kAccBiasF, w1 * -kAccBiasF);
           __syncwarp();
-          *reinterpret_cast<float2*>(sb_s + 2 * lane) = make_float2(fb.x * 0.00390625f, fb.y * 0.00390625f);
-          __syncwarp();
+          if ((g & 1) == 1 && lane == 0) ptx::mbar_arrive(&sh->sc_empty[ss]);
         }
-        const int b = gi % kGroupBufs;
         if (!wait_bounded(&sh->grp_full[b], (gi / kGroupBufs) & 1, abort_flag, p.err, kErrSiteGemmAccFull)) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t base = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * kBN + h * 64;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          uint32_t v[32];
-          ptx::tmem_ld_32x32b_x32(base + half * 32, v);
-          ptx::tmem_wait_ld();
-          if (lowrank) {
-#pragma unroll
-            for (int c = 0; c < 16; ++c)
-              acc[half * 16 + c] = __fadd2_rn(acc[half * 16 + c],
-                                              make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])));
-          } else {
-            const float2 sa2 = make_float2(sa, sa);
-            const float2 nb2 = make_float2(-12582912.f, -12582912.f);
-#pragma unroll
-            for (int c = 0; c < 16; ++c) {
-              const float2 sb2 = *reinterpret_cast<const float2*>(sb_s + half * 32 + 2 * c);
-              const float2 d = __fadd2_rn(make_float2(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1])), nb2);
-              acc[half * 16 + c] = __ffma2_rn(d, __fmul2_rn(sa2, sb2), acc[half * 16 + c]);
-            }
-          }
-          // this half is consumed: preset it again for the buffer's next use
-#pragma unroll
-          for (int c8 = 0; c8 < 4; ++c8) ptx::tmem_st_32x32b_x8_same(base + half * 32 + c8 * 8, kAccBias);
-        }
-        ptx::tmem_wait_st();
+        // both 16-row slabs into registers, then the buffer goes back to the MMA warp
+        uint32_t v[2][32];
+        ptx::tmem_ld_16x256b_x8(base, v[0]);
+        ptx::tmem_ld_16x256b_x8(base + (16u << 16), v[1]);
+        ptx::tmem_wait_ld();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          ptx::mbar_arrive(&sh->grp_empty[b]);
-          if (!lowrank && (g & 1) == 1) ptx::mbar_arrive(&sh->sc_empty[ss]);
+        if (lane == 0) ptx::mbar_arrive(&sh->grp_empty[b]);
+        if (lowrank) {
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              acc[j][i] = __fadd2_rn(acc[j][i], u2f2(v[j >> 1][4 * i + 2 * (j & 1)], v[j >> 1][4 * i + 2 * (j & 1) + 1]));
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) {
+            const float4 s4 = *reinterpret_cast<const float4*>(pr + (4 * i + lc) * 4);
+            const float2 a2 = make_float2(s4.x, s4.y), b2 = make_float2(s4.z, s4.w);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              // s32 256 D + the bits of B is the float B + 256 D exactly (|256 D| < 2^22)
+              const uint32_t* vv = &v[j >> 1][4 * i + 2 * (j & 1)];
+              const float2 vf = u2f2(vv[0] + kAccBias, vv[1] + kAccBias);
+              const float2 tt = __ffma2_rn(vf, a2, b2);
+              acc[j][i] = __ffma2_rn(tt, make_float2(sa[j], sa[j]), acc[j][i]);
+            }
+          }
         }
       }
       sc_it += nk_main;
       if (!ok) break;
-      // Y = acc + bias -> bf16, one 32-row x 64-column box through shared memory and a TMA store
+      // Y = acc + bias -> bf16, one 32-row x 64-column 128B-swizzled box and a TMA store
       if (lane == 0) ptx::bulk_wait_group_read<0>();
       __syncwarp();
 #pragma unroll
-      for (int c8 = 0; c8 < 8; ++c8) {
-        float bv[8];
+      for (int i = 0; i < 8; ++i) {
+        float2 bv = make_float2(0.f, 0.f);
         if (p.bias) {
-          const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + c8 * 8));
-          const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
-#pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            bv[2 * u] = __uint_as_float(bw[u] << 16);
-            bv[2 * u + 1] = __uint_as_float(bw[u] & 0xFFFF0000u);
-          }
-        } else {
-#pragma unroll
-          for (int u = 0; u < 8; ++u) bv[u] = 0.f;
+          const uint32_t bw = __ldg(reinterpret_cast<const unsigned int*>(p.bias + col0 + 8 * i + 2 * lc));
+          bv = make_float2(__uint_as_float(bw << 16), __uint_as_float(bw & 0xFFFF0000u));
         }
-        uint32_t o[4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const float2 a2 = acc[c8 * 4 + u];
-          __nv_bfloat162 hv = __floats2bfloat162_rn(a2.x + bv[2 * u], a2.y + bv[2 * u + 1]);
-          o[u] = *reinterpret_cast<uint32_t*>(&hv);
+        for (int j = 0; j < 4; ++j) {
+          const int row = 8 * j + lr;
+          __nv_bfloat162 hv = __floats2bfloat162_rn(acc[j][i].x + bv.x, acc[j][i].y + bv.y);
+          *reinterpret_cast<__nv_bfloat162*>(buf + row * 128 + ((i ^ (row & 7)) << 4) + lc * 4) = hv;
         }
-        *reinterpret_cast<uint4*>(buf + lane * 128 + ((c8 ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
       }
       ptx::fence_proxy_async_smem();
       __syncwarp();
@@ -440,10 +454,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
-size_t gemm_int4_smem_bytes() {
-  return 1024 + kStages * kStageBytes + kPkStages * kPkStageBytes + kLrBytes + kScStages * kScBytes +
-         kEpiWarps * kEpiBoxBytes + kEpiWarps * 64 * 4 + sizeof(SharedTail);
-}
+size_t gemm_int4_smem_bytes() { return kSmemBytes; }
 
 cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
                              const CUtensorMap& tl2, const CUtensorMap& ty, const CUtensorMap& tsa,

@@ -75,7 +75,7 @@ bool make_tmap_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, uint
 bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows_pad, int64_t K, int g, uint32_t blocks) {
   const uint64_t kblocks = static_cast<uint64_t>(K / (4 * g));
   return make_tmap_3d(m, base, CU_TENSOR_MAP_DATA_TYPE_UINT64, 64, kblocks, static_cast<uint64_t>(rows_pad / 128), 512,
-                      kblocks * 512, 64, static_cast<uint32_t>(256 / (4 * g)), blocks);
+                      kblocks * 512, 64, static_cast<uint32_t>(2 * 256 / (4 * g)), blocks);
 }
 
 int device_sm_count() {
@@ -265,8 +265,20 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
     p.tiles_n = static_cast<int>((N + 255) / 256);
     p.num_tiles = p.tiles_m * p.tiles_n;
     CUtensorMap ta, tb, tsfa, tsfb;
-    if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) return SVDQ_ERR_CUDA;
-    if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) return SVDQ_ERR_CUDA;
+    // K a multiple of 256: each operand load covers two K steps (a 3-D view of the rows as
+    // [K/256 chunks][rows][128 bytes]); otherwise two 2-D loads per slot
+    p.op_pair = (K % 256) == 0 ? 1 : 0;
+    if (p.op_pair) {
+      if (!make_tmap_3d(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, M, K / 256, K / 2, 128, 128, 128, 2,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
+      if (!make_tmap_3d(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 128, N, K / 256, K / 2, 128, 128, 128, 2,
+                        CU_TENSOR_MAP_SWIZZLE_128B))
+        return SVDQ_ERR_CUDA;
+    } else {
+      if (!make_tmap(&ta, a_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, M, 128, 128)) return SVDQ_ERR_CUDA;
+      if (!make_tmap(&tb, w_codes, CU_TENSOR_MAP_DATA_TYPE_UINT8, 1, K / 2, N, 128, 128)) return SVDQ_ERR_CUDA;
+    }
     if (!make_tmap_sf(&tsfa, a_scales, p.Mpad, K, g, 1)) return SVDQ_ERR_CUDA;
     if (!make_tmap_sf(&tsfb, w_scales, p.Npad, K, g, 2)) return SVDQ_ERR_CUDA;
     if (rank > 0) {
@@ -276,9 +288,7 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
       tz = ta;
       tl2 = tb;
     }
-    CUtensorMap ty;
-    if (!make_tmap(&ty, Y_bf16, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, N, M, 64, 32)) return SVDQ_ERR_CUDA;
-    e = launch_gemm_fp4(fmt == SVDQ_FMT_MXFP4_G32, ta, tb, tsfa, tsfb, tz, tl2, ty, p, sms,
+    e = launch_gemm_fp4(fmt == SVDQ_FMT_MXFP4_G32, ta, tb, tsfa, tsfb, tz, tl2, p, sms,
                         static_cast<cudaStream_t>(cuda_stream));
   } else if (fmt == SVDQ_FMT_W8A8) {
     p.tiles_m = static_cast<int>((M + 255) / 256);

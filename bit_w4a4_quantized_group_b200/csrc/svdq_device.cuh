@@ -29,7 +29,34 @@ enum : int {
   kErrSiteGemmConvDone = 19,
   kErrSiteGemmAccFinal = 20,
   kErrSiteSelftest = 90,
+  // Debug builds (-DSVDQ_DEBUG) only: an access outside its buffer was found and skipped.
+  kErrSiteBoundsGlobal = 201,   // a plain global load or store past its buffer
+  kErrSiteBoundsShared = 202,   // a shared-memory access past the dynamic allocation
 };
+
+// Bounds checks of the debug build.  SVDQ_DEBUG_OK(cond, site, err) is true in a release build
+// (the check compiles away); in a debug build a false condition records `site` in the device
+// error word (first failure wins) and the caller skips the access, so a bad index never turns
+// into an out-of-bounds access.
+#ifdef SVDQ_DEBUG
+__device__ __forceinline__ bool debug_in_bounds(bool ok, int site, int* err) {
+  if (!ok) atomicCAS(err, 0, site);
+  return ok;
+}
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+  uint32_t v;
+  asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(v));
+  return v;
+}
+// [p, p + bytes) lies inside this CTA's dynamic shared memory starting at base
+__device__ __forceinline__ bool smem_in_bounds(const void* base, const void* p, uint32_t bytes) {
+  const uintptr_t b = reinterpret_cast<uintptr_t>(base), a = reinterpret_cast<uintptr_t>(p);
+  return a >= b && a + bytes <= b + dynamic_smem_bytes();
+}
+#define SVDQ_DEBUG_OK(cond, site, err) (::svdq::debug_in_bounds((cond), (site), (err)))
+#else
+#define SVDQ_DEBUG_OK(cond, site, err) (true)
+#endif
 
 // A wait gives up after this many nanoseconds (~1 s); legitimate waits here
 // last microseconds.
@@ -104,6 +131,7 @@ struct GemmParams {
   __nv_bfloat16* Y;          // [M][N]
   int* err;
   int num_tiles, tiles_m, tiles_n;
+  int op_pair;               // FP4: A and B tensor maps are 3-D and load two K steps at once
 };
 
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
@@ -112,7 +140,7 @@ cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& t
 // NVFP4 (mx = false) or MXFP4 (mx = true) GEMM with the fused low-rank up projection.
 cudaError_t launch_gemm_fp4(bool mx, const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tsfa,
                             const CUtensorMap& tsfb, const CUtensorMap& tz, const CUtensorMap& tl2,
-                            const CUtensorMap& ty, const GemmParams& p, int num_sms, cudaStream_t s);
+                            const GemmParams& p, int num_sms, cudaStream_t s);
 size_t gemm_int4_smem_bytes();
 // W8A8 GEMM: s32 accumulation of the 8-bit product, per-row / per-column fp32 scales in the
 // epilogue, the low-rank product in a second (fp32) TMEM accumulator.

@@ -32,11 +32,17 @@
  *   - Errors: launch failures map to SVDQ_ERR_CUDA.  Every wait inside the
  *     kernels is bounded; a wait that runs out records SVDQ_ERR_TIMEOUT in the
  *     device error word and the kernel returns early (read it with
- *     svdq_get_last_device_error).  NaN / Inf inputs are outside the contract.
+ *     svdq_get_last_device_error).  After SVDQ_ERR_TIMEOUT the outputs of the
+ *     calls that ran since the error word was last cleared are undefined: the
+ *     kernel stopped before writing all of them.  NaN / Inf inputs are outside
+ *     the contract.
  *
  * Buffer layouts (all row-major, little-endian)
  *   X        bf16 [M][K]
- *   lambda   fp32 [K]                    (NULL means lambda = 1)
+ *   lambda   fp32 [K]                    (NULL means lambda = 1); every entry finite,
+ *                                        normal and > 0 (the divide assumes a normal
+ *                                        positive divisor; other values are outside
+ *                                        the contract)
  *   L1       bf16 [r][K]                 (the "l1 = V^T" [rank, in] shape)
  *   Z        bf16 [M][r]                 Z = bf16(X_hat L1^T), fp32 accumulation
  *   L2s      bf16 [N][r]                 (the "l2 = U S" [out, rank] shape), stored
