@@ -43,8 +43,9 @@
 //     single multiply by g_x g_w scales both terms and Y is written once;
 //   * eight epilogue warps per CTA drain TMEM (tcgen05.ld) into registers and
 //     release the accumulator at once, then apply g_x g_w and the bias and store
-//     bf16 Y from registers (each thread 256 contiguous bytes of its row), while
-//     the next tile's MMAs run.
+//     bf16 Y from registers while the next tile's MMAs run: each thread writes
+//     256 contiguous bytes of its row with 32-byte (one sector) stores, which
+//     halves the write requests of 16-byte stores (32 rows per warp instruction).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -396,35 +397,46 @@ __global__ void __launch_bounds__(kThreads, 1)
       acc_ph ^= 1u;
       if (!active) continue;
       // Y = g_x g_w * acc + bias -> bf16, written straight from registers: each thread
-      // stores its row's 128 columns (256 contiguous bytes); rows past M are skipped.
+      // stores its row's 128 columns (256 contiguous bytes), 32 bytes (one sector) per store
+      // when Y is 32-byte aligned; rows past M are skipped.
       const int row = m0 + q * 32 + lane;
       if (row >= p.M) continue;
       __nv_bfloat16* yrow = p.Y + static_cast<size_t>(row) * p.N + col0;
 #pragma unroll
-      for (int c8 = 0; c8 < 16; ++c8) {
-        const int cl = c8 * 8;                               // column within this warp's 128
-        float bv[8];
-        if (p.bias) {
-          const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + cl));
-          const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+      for (int c16 = 0; c16 < 8; ++c16) {
+        const int cl = c16 * 16;                             // column within this warp's 128
+        float bv[16];
+        const bool in_n = SVDQ_IN_GLOBAL(col0 + cl + 16 <= p.N, p.err);
+        if (p.bias && in_n) {
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            bv[2 * e] = __uint_as_float(bw[e] << 16);
-            bv[2 * e + 1] = __uint_as_float(bw[e] & 0xFFFF0000u);
+          for (int hb = 0; hb < 2; ++hb) {
+            const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + cl + 8 * hb));
+            const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              bv[8 * hb + 2 * e] = __uint_as_float(bw[e] << 16);
+              bv[8 * hb + 2 * e + 1] = __uint_as_float(bw[e] & 0xFFFF0000u);
+            }
           }
         } else {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) bv[e] = 0.f;
+          for (int e = 0; e < 16; ++e) bv[e] = 0.f;
         }
-        uint32_t o[4];
+        uint32_t o[8];
 #pragma unroll
-        for (int e = 0; e < 4; ++e) {
+        for (int e = 0; e < 8; ++e) {
           const float y0 = fmaf(__uint_as_float(v[cl / 32][cl % 32 + 2 * e]), sc, bv[2 * e]);
           const float y1 = fmaf(__uint_as_float(v[cl / 32][cl % 32 + 2 * e + 1]), sc, bv[2 * e + 1]);
           __nv_bfloat162 hv = __floats2bfloat162_rn(y0, y1);
           o[e] = *reinterpret_cast<uint32_t*>(&hv);
         }
-        *reinterpret_cast<uint4*>(yrow + cl) = make_uint4(o[0], o[1], o[2], o[3]);
+        if (!in_n) {
+        } else if (p.y_align32) {
+          ptx::st_global_v8(yrow + cl, o);
+        } else {
+          *reinterpret_cast<uint4*>(yrow + cl) = make_uint4(o[0], o[1], o[2], o[3]);
+          *reinterpret_cast<uint4*>(yrow + cl + 8) = make_uint4(o[4], o[5], o[6], o[7]);
+        }
       }
     }
   }

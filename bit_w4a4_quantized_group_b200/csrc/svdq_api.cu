@@ -254,6 +254,7 @@ extern "C" svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int
   p.w_scales = static_cast<const uint8_t*>(w_scales);
   p.bias = static_cast<const __nv_bfloat16*>(bias_bf16);
   p.Y = static_cast<__nv_bfloat16*>(Y_bf16);
+  p.y_align32 = (reinterpret_cast<uintptr_t>(Y_bf16) & 31u) == 0 ? 1 : 0;
   p.err = device_error_word();
   if (!p.err) return SVDQ_ERR_CUDA;
 

@@ -57,6 +57,11 @@ __device__ __forceinline__ bool smem_in_bounds(const void* base, const void* p, 
 #else
 #define SVDQ_DEBUG_OK(cond, site, err) (true)
 #endif
+// A plain global access whose index satisfies `cond`; a shared-memory access of `bytes` at
+// `ptr` inside the dynamic allocation that starts at `base`.
+#define SVDQ_IN_GLOBAL(cond, err) SVDQ_DEBUG_OK((cond), ::svdq::kErrSiteBoundsGlobal, (err))
+#define SVDQ_IN_SMEM(base, ptr, bytes, err) \
+  SVDQ_DEBUG_OK(::svdq::smem_in_bounds((base), (ptr), (bytes)), ::svdq::kErrSiteBoundsShared, (err))
 
 // A wait gives up after this many nanoseconds (~1 s); legitimate waits here
 // last microseconds.
@@ -132,6 +137,7 @@ struct GemmParams {
   int* err;
   int num_tiles, tiles_m, tiles_n;
   int op_pair;               // FP4: A and B tensor maps are 3-D and load two K steps at once
+  int y_align32;             // Y is 32-byte aligned (256-bit stores)
 };
 
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,

@@ -76,15 +76,18 @@ def codes_bytes(fmt, codes: np.ndarray) -> np.ndarray:
     return pack_codes_bytes(codes)
 
 
-def run_gemm(fmt, M, N, K, rank, a_codes, a_scales, gx, w_codes, w_scales, gw, Z, L2s, bias):
-    """All operand arguments are host NumPy buffers in library layout (or device tensors)."""
+def run_gemm(fmt, M, N, K, rank, a_codes, a_scales, gx, w_codes, w_scales, gw, Z, L2s, bias, y_offset=0):
+    """All operand arguments are host NumPy buffers in library layout (or device tensors).
+    y_offset: Y starts that many bf16 elements into a larger buffer (8: 16-byte but not
+    32-byte aligned)."""
     def d(x):
         if x is None:
             return None
         if isinstance(x, torch.Tensor):
             return x
         return torch.from_numpy(np.ascontiguousarray(x)).cuda()
-    Y = torch.full((M, N), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Ybuf = torch.full((M * N + y_offset,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    Y = Ybuf[y_offset:].view(M, N)
     B.w4a4_gemm_lowrank_up_t(fmt, M, N, K, rank, d(a_codes), d(a_scales), gx, d(w_codes), d(w_scales), gw,
                              None if rank == 0 else (Z if isinstance(Z, torch.Tensor) else dev_bf16(Z)),
                              None if rank == 0 else (L2s if isinstance(L2s, torch.Tensor) else dev_bf16(L2s)),

@@ -148,7 +148,7 @@ def test_prologue_rounding_ties_int4():
     _check_prologue("int4", X, None, 1.0, None)
 
 
-def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
+def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True, y_offset=0):
     layer, prep = _layer(M, K, N, rank, seed=seed, fmt=fmt)
     gx = prep["act_gscale"]
     packed = O.pack_weight(fmt, prep["R_nk"], prep["L1_rk"], prep["L2_nr"], gx)
@@ -158,7 +158,7 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True):
     Y = run_gemm(fmt, M, N, K, rank,
                  codes_bytes(fmt, pro["q"]["codes"]), encode_scales(fmt, pro["q"]["scale_bits"], M, K), gx,
                  codes_bytes(fmt, packed["q"]["codes"]), encode_scales(fmt, packed["q"]["scale_bits"], N, K),
-                 packed["gscale"], pro["Z"], packed["L2_scaled"], bias)
+                 packed["gscale"], pro["Z"], packed["L2_scaled"], bias, y_offset=y_offset)
     Yg = host_bf16(Y)
     assert np.all(np.isfinite(Yg))
     e_ref = rel_fro(Yg, ref["Y"])
@@ -184,6 +184,13 @@ def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
     """More output tiles than resident CTAs (clusters), so each persistent CTA drains several
     accumulators; short K (one to three pipeline steps per tile) and a two-step branch."""
     _gemm_case(fmt, M, N, K, rank, seed=5 + M + K + rank)
+
+
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
+def test_gemm_parity_y_not_32_byte_aligned(fmt):
+    """Y 16-byte but not 32-byte aligned: the FP4 epilogue falls back from 32-byte to
+    16-byte stores (and a ragged M keeps the row guard in play)."""
+    _gemm_case(fmt, 300, 640, 512, 32, seed=23, y_offset=8)
 
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
