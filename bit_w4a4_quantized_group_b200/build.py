@@ -1,10 +1,16 @@
 """Build libsvdq.so (sm_100a) in-tree with nvcc.
 
-    python -m bit_w4a4_quantized_group_b200.build [--verbose]
+    python -m bit_w4a4_quantized_group_b200.build [--verbose] [--debug]
 
 Each source under ``csrc/`` is compiled to an object in ``_build/`` (in
 parallel), then linked into ``_lib/libsvdq.so`` with the CUDA runtime linked
 statically.  No GPU is needed to build.
+
+``--debug`` builds ``_lib/libsvdq_debug.so`` instead (objects in ``_build_debug/``):
+the same kernels compiled with -DSVDQ_DEBUG, in which every plain global or
+shared-memory access of the kernels checks its index first; an access that
+would fall outside its buffer is skipped and recorded in the device error word
+(sites 201 and 202 of svdq_get_last_device_error).
 """
 from __future__ import annotations
 
@@ -21,6 +27,8 @@ INCLUDE = os.path.join(ROOT, "include")
 BUILD = os.path.join(PKG, "_build")
 LIBDIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIBDIR, "libsvdq.so")
+BUILD_DEBUG = os.path.join(PKG, "_build_debug")
+LIB_DEBUG = os.path.join(LIBDIR, "libsvdq_debug.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 COMMON = ["-O3", "-std=c++17", "-Xcompiler", "-fPIC", "-I", INCLUDE, "-I", CSRC]
@@ -49,9 +57,9 @@ def _deps_mtime():
     return m
 
 
-def _compile(src: str, verbose: bool) -> str:
-    obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    cmd = [nvcc(), *ARCH, *COMMON, "-c", src, "-o", obj]
+def _compile(src: str, verbose: bool, debug: bool = False) -> str:
+    obj = os.path.join(BUILD_DEBUG if debug else BUILD, os.path.basename(src) + ".o")
+    cmd = [nvcc(), *ARCH, *COMMON, *(["-DSVDQ_DEBUG"] if debug else []), "-c", src, "-o", obj]
     if src.endswith(".cu"):
         cmd += ["-lineinfo"]
         if verbose:
@@ -66,23 +74,25 @@ def _compile(src: str, verbose: bool) -> str:
     return obj
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    """Compile every CUDA / C++ source of the library for sm_100a; return the .so path."""
-    if (not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _deps_mtime()):
-        return LIB
-    os.makedirs(BUILD, exist_ok=True)
+def build(force: bool = False, verbose: bool = False, debug: bool = False) -> str:
+    """Compile every CUDA / C++ source of the library for sm_100a; return the .so path
+    (the bounds-checking debug library when debug is true)."""
+    lib = LIB_DEBUG if debug else LIB
+    if (not force and os.path.exists(lib) and os.path.getmtime(lib) >= _deps_mtime()):
+        return lib
+    os.makedirs(BUILD_DEBUG if debug else BUILD, exist_ok=True)
     os.makedirs(LIBDIR, exist_ok=True)
     srcs = _sources()
     with cf.ThreadPoolExecutor(max_workers=min(8, len(srcs))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose), srcs))
-    tmp = LIB + ".tmp"
+        objs = list(ex.map(lambda s: _compile(s, verbose, debug), srcs))
+    tmp = lib + ".tmp"
     cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
     r = subprocess.run(cmd, capture_output=True, text=True)
     if r.returncode != 0:
         raise RuntimeError(f"link failed:\n{r.stdout}\n{r.stderr}")
-    os.replace(tmp, LIB)
-    return LIB
+    os.replace(tmp, lib)
+    return lib
 
 
 if __name__ == "__main__":
-    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv))
+    print(build(force="--force" in sys.argv, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

@@ -226,10 +226,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint8_t* pa = pk_smem + ps * kPkStageBytes + r * 64;
           const uint8_t* pb = pa + kPkOpBytes;
           const int sw = (r >> 1) & 3;
+          const bool in_s = SVDQ_IN_SMEM(smem_raw, pa, 64, p.err) && SVDQ_IN_SMEM(smem_raw, pb, 64, p.err);
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            va[h][i] = *reinterpret_cast<const uint4*>(pa + ((i ^ sw) << 4));
-            vb[h][i] = *reinterpret_cast<const uint4*>(pb + ((i ^ sw) << 4));
+            va[h][i] = in_s ? *reinterpret_cast<const uint4*>(pa + ((i ^ sw) << 4)) : make_uint4(0, 0, 0, 0);
+            vb[h][i] = in_s ? *reinterpret_cast<const uint4*>(pb + ((i ^ sw) << 4)) : make_uint4(0, 0, 0, 0);
           }
         }
         ptx::mbar_arrive(&sh->pk_empty[ps]);
@@ -242,6 +243,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int r = threadIdx.x + 64 * h;
           uint8_t* arow_s = smem + s * kStageBytes + r * 128;
           uint8_t* brow_s = arow_s + kOpBytes;
+          if (!(SVDQ_IN_SMEM(smem_raw, arow_s, 128, p.err) && SVDQ_IN_SMEM(smem_raw, brow_s, 128, p.err))) continue;
           // 64 packed bytes -> 128 int8 bytes = 8 chunks of 16 bytes, 128B-swizzled by row
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
@@ -369,13 +371,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint8_t* sc = sc_smem + ss * kScBytes + (g & 1) * 256;
+          if (SVDQ_IN_SMEM(smem_raw, sc, 256, p.err) && SVDQ_IN_SMEM(smem_raw, sc + 512, 256, p.err) &&
+              SVDQ_IN_SMEM(smem_raw, pairs + (g & 1) * 128 + lane * 4, 16, p.err)) {
 #pragma unroll
-          for (int j = 0; j < 4; ++j)
-            sa[j] = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + 8 * j + lr) * 2));
-          const float2 sw = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
-          const float w0 = sw.x * 0.00390625f, w1 = sw.y * 0.00390625f;
-          *reinterpret_cast<float4*>(pairs + (g & 1) * 128 + lane * 4) =
-              make_float4(w0, w1, w0 * -kAccBiasF, w1 * -kAccBiasF);
+            for (int j = 0; j < 4; ++j)
+              sa[j] = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + 8 * j + lr) * 2));
+            const float2 sw = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
+            const float w0 = sw.x * 0.00390625f, w1 = sw.y * 0.00390625f;
+            *reinterpret_cast<float4*>(pairs + (g & 1) * 128 + lane * 4) =
+                make_float4(w0, w1, w0 * -kAccBiasF, w1 * -kAccBiasF);
+          }
           __syncwarp();
           if ((g & 1) == 1 && lane == 0) ptx::mbar_arrive(&sh->sc_empty[ss]);
         }
@@ -401,7 +406,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 s4 = *reinterpret_cast<const float4*>(pr + (4 * i + lc) * 4);
+            const float4 s4 = SVDQ_IN_SMEM(smem_raw, pr + (4 * i + lc) * 4, 16, p.err)
+                                  ? *reinterpret_cast<const float4*>(pr + (4 * i + lc) * 4)
+                                  : make_float4(0.f, 0.f, 0.f, 0.f);
             const float2 a2 = make_float2(s4.x, s4.y), b2 = make_float2(s4.z, s4.w);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -422,7 +429,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float2 bv = make_float2(0.f, 0.f);
-        if (p.bias) {
+        if (p.bias && SVDQ_IN_GLOBAL(col0 + 8 * i + 2 * lc + 2 <= p.N, p.err)) {
           const uint32_t bw = __ldg(reinterpret_cast<const unsigned int*>(p.bias + col0 + 8 * i + 2 * lc));
           bv = make_float2(__uint_as_float(bw << 16), __uint_as_float(bw & 0xFFFF0000u));
         }
@@ -430,7 +437,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int j = 0; j < 4; ++j) {
           const int row = 8 * j + lr;
           __nv_bfloat162 hv = __floats2bfloat162_rn(acc[j][i].x + bv.x, acc[j][i].y + bv.y);
-          *reinterpret_cast<__nv_bfloat162*>(buf + row * 128 + ((i ^ (row & 7)) << 4) + lc * 4) = hv;
+          if (SVDQ_IN_SMEM(smem_raw, buf + row * 128 + ((i ^ (row & 7)) << 4) + lc * 4, 4, p.err))
+            *reinterpret_cast<__nv_bfloat162*>(buf + row * 128 + ((i ^ (row & 7)) << 4) + lc * 4) = hv;
         }
       }
       ptx::fence_proxy_async_smem();

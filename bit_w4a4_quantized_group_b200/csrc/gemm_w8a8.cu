@@ -238,7 +238,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int m0 = tiles.mb(j) * kBM + static_cast<int>(rank) * kRows;
       const int col0 = tiles.nb(j) * kBN + h * 128;
       const int row = m0 + q * 32 + lane;
-      const bool active = col0 < p.N;          // the second half of a last tile may lie past N
+      const bool active = col0 < p.N &&        // the second half of a last tile may lie past N
+                          SVDQ_IN_GLOBAL(col0 + 128 <= p.N, p.err);
       const float sx = row < p.Mpad ? __ldg(sx_all + row) : 0.f;
       const uint32_t base = tmem + (static_cast<uint32_t>(q * 32) << 16) + b * 256 + h * 128;
       if (!wait_bounded(&sh->acc_full[b], par, abort_flag, p.err, kErrSiteGemmAccFull)) break;
@@ -310,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int c8 = 0; c8 < 4; ++c8) {
             const int cl = c2 * 32 + c8 * 8;          // column within the 64-column box
             float bv[8];
-            if (p.bias) {
+            if (p.bias && SVDQ_IN_GLOBAL(col0 + box * 64 + cl + 8 <= p.N, p.err)) {
               const uint4 braw = __ldg(reinterpret_cast<const uint4*>(p.bias + col0 + box * 64 + cl));
               const uint32_t bw[4] = {braw.x, braw.y, braw.z, braw.w};
 #pragma unroll
@@ -329,7 +330,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               o[e] = *reinterpret_cast<uint32_t*>(&hv);
             }
             const int chunk = cl / 8;                 // 16-byte chunk of the 128-byte row
-            *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
+            if (SVDQ_IN_SMEM(smem_raw, buf + lane * 128 + ((chunk ^ (lane & 7)) << 4), 16, p.err))
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((chunk ^ (lane & 7)) << 4)) = make_uint4(o[0], o[1], o[2], o[3]);
           }
         }
         ptx::fence_proxy_async_smem();

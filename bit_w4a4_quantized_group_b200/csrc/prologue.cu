@@ -210,6 +210,10 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) cur[i] = lv[i];
       if (it + 1 < nit) load_lambda(kbeg + (kt0 + (it + 1) % nkt) % nkt);
+      if (!(SVDQ_IN_SMEM(smem_raw, lam_s, BK * 4, p.err) && SVDQ_IN_SMEM(smem_raw, rlam_s, BK * 4, p.err))) {
+        ptx::mbar_arrive(&full[s]);
+        continue;
+      }
 #pragma unroll
       for (int i = 0; i < BK / 32; ++i) {
         lam_s[i * 32 + lane] = cur[i];
@@ -247,7 +251,12 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       if (!wait_bounded(&full[s], ph, abort_flag, p.err, kErrSiteProFull)) { ok = false; break; }
       const int kt = kbeg + (kt0 + ki) % nkt;
       const int col0 = kt * BK + phase * 64;
-      if (col0 < p.K) {
+      if (col0 < p.K &&
+          SVDQ_IN_SMEM(smem_raw, smem + s * L.stage_bytes + L.x_off + phase * kXBoxBytes, kXBoxBytes, p.err) &&
+          (RANK == 0 || SVDQ_IN_SMEM(smem_raw, smem + s * L.stage_bytes + L.l1_off + phase * 128 * RANK, 128 * RANK, p.err)) &&
+          SVDQ_IN_SMEM(smem_raw, smem + s * L.stage_bytes + L.lam_off + phase * 256, 256, p.err) &&
+          SVDQ_IN_SMEM(smem_raw, smem + s * L.stage_bytes + L.rlam_off + phase * 256, 256, p.err) &&
+          SVDQ_IN_SMEM(smem_raw, cst, CSTB, p.err)) {
         const uint8_t* st = smem + s * L.stage_bytes;
         const uint32_t xbox = ptx::smem_u32(st + L.x_off + phase * kXBoxBytes);
         const uint32_t l1box = ptx::smem_u32(st + L.l1_off + phase * 128 * RANK);
@@ -371,8 +380,11 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
                               (row_a % 32) * 16 + ((row_a % 128) / 32) * 4 + grp % 4;
             const size_t bb = (static_cast<size_t>(row_b / 128) * (p.K / 128) + grp / 4) * 512 +
                               (row_b % 32) * 16 + ((row_b % 128) / 32) * 4 + grp % 4;
-            *reinterpret_cast<uint16_t*>(sc + ba) = static_cast<uint16_t>(sb_a);
-            *reinterpret_cast<uint16_t*>(sc + bb) = static_cast<uint16_t>(sb_b);
+            const size_t nsc = static_cast<size_t>(p.Mpad) * (p.K / 32);
+            if (SVDQ_IN_GLOBAL(ba + 2 <= nsc && bb + 2 <= nsc, p.err)) {
+              *reinterpret_cast<uint16_t*>(sc + ba) = static_cast<uint16_t>(sb_a);
+              *reinterpret_cast<uint16_t*>(sc + bb) = static_cast<uint16_t>(sb_b);
+            }
           }
         } else if (FMT == kFmtInt4) {
           // one 64-element group per row per box
@@ -418,8 +430,10 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           if (tig == 0) {
             const int grp = col0 / 64;
             __half* sc = reinterpret_cast<__half*>(p.scales);
-            sc[static_cast<size_t>(grp) * p.Mpad + row_a] = ha;
-            sc[static_cast<size_t>(grp) * p.Mpad + row_b] = hb;
+            if (SVDQ_IN_GLOBAL(grp < p.K / 64 && row_b < p.Mpad, p.err)) {
+              sc[static_cast<size_t>(grp) * p.Mpad + row_a] = ha;
+              sc[static_cast<size_t>(grp) * p.Mpad + row_b] = hb;
+            }
           }
         } else if (FMT == kFmtW8a8) {
           if (pass == 0) {
@@ -462,8 +476,11 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
                               (row_a % 32) * 16 + ((row_a % 128) / 32) * 4;
             const size_t bb = (static_cast<size_t>(row_b / 128) * (p.K / 64) + grp4) * 512 +
                               (row_b % 32) * 16 + ((row_b % 128) / 32) * 4;
-            *reinterpret_cast<uint32_t*>(sc + ba) = sc_pack_a;
-            *reinterpret_cast<uint32_t*>(sc + bb) = sc_pack_b;
+            const size_t nsc = static_cast<size_t>(p.Mpad) * (p.K / 16);
+            if (SVDQ_IN_GLOBAL(ba + 4 <= nsc && bb + 4 <= nsc, p.err)) {
+              *reinterpret_cast<uint32_t*>(sc + ba) = sc_pack_a;
+              *reinterpret_cast<uint32_t*>(sc + bb) = sc_pack_b;
+            }
           }
         }
         __syncwarp();
@@ -472,14 +489,15 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
           const int r = lane >> 1, h = lane & 1;
           const int row = m0 + strip * 16 + r;
           const uint4 v = *reinterpret_cast<const uint4*>(cst + r * 32 + h * 16);
-          if (row < p.M) *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * K2 + col0 / 2 + h * 16) = v;
+          if (row < p.M && SVDQ_IN_GLOBAL(col0 / 2 + h * 16 + 16 <= K2, p.err))
+            *reinterpret_cast<uint4*>(p.codes + static_cast<size_t>(row) * K2 + col0 / 2 + h * 16) = v;
         } else if (pass == 1) {
           // 16 rows x 64 bytes of 8-bit codes -> global, two 16-byte segments per lane
           const int r = lane >> 1, h = lane & 1;
           const int row = m0 + strip * 16 + r;
           const uint4 v0 = *reinterpret_cast<const uint4*>(cst + r * 64 + h * 32);
           const uint4 v1 = *reinterpret_cast<const uint4*>(cst + r * 64 + h * 32 + 16);
-          if (row < p.M) {
+          if (row < p.M && SVDQ_IN_GLOBAL(col0 + h * 32 + 32 <= p.K, p.err)) {
             uint8_t* dst = p.codes + static_cast<size_t>(row) * p.K + col0 + h * 32;
             *reinterpret_cast<uint4*>(dst) = v0;
             *reinterpret_cast<uint4*>(dst + 16) = v1;
@@ -496,7 +514,7 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       rmax_b = fmaxf(rmax_b, __shfl_xor_sync(0xffffffffu, rmax_b, 1));
       rmax_a = fmaxf(rmax_a, __shfl_xor_sync(0xffffffffu, rmax_a, 2));
       rmax_b = fmaxf(rmax_b, __shfl_xor_sync(0xffffffffu, rmax_b, 2));
-      if (tig == 0) {
+      if (tig == 0 && SVDQ_IN_SMEM(smem_raw, rmax_s + (phase * 2 + strip) * 16, 64, p.err)) {
         rmax_s[(phase * 2 + strip) * 16 + g] = rmax_a;
         rmax_s[(phase * 2 + strip) * 16 + g + 8] = rmax_b;
       }
@@ -513,8 +531,10 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       const float sb = __double2float_rn(__ddiv_rn(static_cast<double>(amax_b), 127.0));
       if (phase == 0 && tig == 0) {
         float* sc = reinterpret_cast<float*>(p.scales);
-        sc[row_a] = sa;             // rows up to Mpad; rows past M read zeros and get 0
-        sc[row_b] = sb;
+        if (SVDQ_IN_GLOBAL(row_b < p.Mpad, p.err)) {
+          sc[row_a] = sa;             // rows up to Mpad; rows past M read zeros and get 0
+          sc[row_b] = sb;
+        }
       }
       w8_fa = sa < 0x1p-64f ? 0x1p64f : 1.f;
       w8_fb = sb < 0x1p-64f ? 0x1p64f : 1.f;
@@ -530,8 +550,9 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       named_barrier_sync(1, 32 * NW);
       float* zbuf = reinterpret_cast<float*>(smem);       // [phase][strip][16][RANK]
       float* zb = zbuf + ((phase * 2 + strip) * 16) * RANK;
+      const bool zb_ok = SVDQ_IN_SMEM(smem_raw, zb, 16 * RANK * 4, p.err);
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
+      for (int nt = 0; nt < (zb_ok ? NT : 0); ++nt) {
         const int c = nt * 8 + tig * 2;
         zb[g * RANK + c] = acc[nt][0];
         zb[g * RANK + c + 1] = acc[nt][1];
