@@ -753,7 +753,10 @@ def main():
         "lowrank_overhead_pct": 100.0 * (t_gemm / t_gemm0 - 1.0),
         "gemm_frac_fp4_peak": (flops / t_gemm / 1e12) / peak,
         "prologue": {"bound": "hbm", "GB/s": pro_bytes / t_pro / 1e9, "peak": hbm,
-                     "frac": pro_bytes / t_pro / 1e9 / hbm, "bytes": pro_bytes},
+                     "frac": pro_bytes / t_pro / 1e9 / hbm, "bytes": pro_bytes,
+                     "traffic": recorded_traffic(os.path.join(ROOT, "bit_w4a4_quantized_group_b200", "csrc",
+                                                              "prologue.cu"),
+                                                 f"prologue_{cfg.name}_{fmt}_r{r}")},
         "fusion": None if not fusion else {
             "layer_r0_us": t_r0 * 1e6, "fused_layer_us": t_step * 1e6,
             "fused_overhead_pct": 100.0 * (t_step / t_r0 - 1.0),
