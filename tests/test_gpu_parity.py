@@ -186,6 +186,15 @@ def test_gemm_parity_many_tiles_per_cta(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=5 + M + K + rank)
 
 
+@pytest.mark.parametrize("fmt", ["nvfp4", "mxfp4"])
+@pytest.mark.parametrize("M,N,K,rank", [(200, 384, 3072, 32), (256, 512, 2048, 0), (1, 256, 1024, 128),
+                                        (129, 768, 6144, 16)])
+def test_gemm_parity_few_tiles(fmt, M, N, K, rank):
+    """Few tiles with long K (one to three tiles on the whole GPU): ragged M, a half tile past
+    N, rank 0 and a long branch."""
+    _gemm_case(fmt, M, N, K, rank, seed=29 + M + K + rank)
+
+
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 def test_gemm_parity_y_not_32_byte_aligned(fmt):
     """Y 16-byte but not 32-byte aligned: the FP4 epilogue falls back from 32-byte to
