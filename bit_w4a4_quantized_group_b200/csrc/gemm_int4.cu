@@ -19,19 +19,20 @@
 //     8-element chunk, identically for A and B, which leaves each group's dot
 //     product unchanged;
 //   * the MMA warp issues tcgen05 kind::i8 MMAs (s8 x s8 -> s32) per 64-element
-//     group into one of four TMEM group buffers.  Each buffer is preset to the
-//     bit pattern of the float B = 1.5 * 2^23, so after the MMAs it holds the fp32
-//     number v = B + 256 D_g exactly (|256 D_g| <= 2^20);
-//   * eight epilogue warps (two per TMEM lane quarter, 64 columns each) drain
-//     each group buffer with two 32-column loads, preset it again while they
-//     scale the values, and hand it back; the group's scales are prepared before
-//     its product is waited for.
-//     The scaling takes two fp32 FMAs per element and group:
+//     group into one of four TMEM group buffers (the group's first MMA overwrites
+//     the buffer with 256 D_g);
+//   * the widening warps also turn each K step's fp16 group scales into fp32 once,
+//     s_w/256 per column and s_x per row for both groups, in a ring of their own, so
+//     that no epilogue warp converts scales;
+//   * eight epilogue warps (two per TMEM lane quarter, 64 columns each) read each
+//     group buffer in the 16x256b shape (4 rows x 16 columns per thread) and hand
+//     it back at once.  Adding the bits of B = 1.5 * 2^23 to the s32 value gives
+//     the fp32 number v = B + 256 D_g exactly (|256 D_g| < 2^22).  The scaling then
+//     takes two fp32 FMAs per element and group:
 //        t = fma(v, s_w/256, -B s_w/256) = RN(D_g s_w)  (B s_w/256 is exact, and
 //            the fma rounds v s_w/256 - B s_w/256 = D_g s_w once),
 //        acc = fma(t, s_x, acc),
-//     packed two columns at a time (f32x2); the per-column pairs (s_w/256,
-//     -B s_w/256) come from shared memory as one 16-byte broadcast per two columns;
+//     packed two columns at a time (f32x2);
 //   * the low-rank branch is one more "group" (bf16 kind::f16 MMAs, added as is)
 //     whose Z and L2 tiles the producer loads with TMA into their own slot;
 //   * Y leaves through 128B-swizzled 32 x 64 shared-memory boxes and TMA stores.
@@ -62,10 +63,11 @@ constexpr uint32_t kStageBytes = 2 * kOpBytes; // A then B
 constexpr uint32_t kPkOpBytes = kBM * 64;      // 8 KB: 128 rows x 64 packed bytes
 constexpr uint32_t kPkStageBytes = 2 * kPkOpBytes;
 constexpr uint32_t kLrBytes = 2 * kOpBytes;    // Z tile + L2 tile (bf16, 64 columns)
-constexpr int kScStages = 8;                   // group-scale ring, one slot per K step
+constexpr int kScStages = 3;                   // fp16 group-scale ring (TMA), one slot per K step
+constexpr int kCvtStages = 6;                  // fp32 scale ring (widening warps -> epilogue), one slot per K step
+constexpr uint32_t kCvtBytes = 2048;           // s_w / 256: 2 groups x 128 columns, s_x: 2 groups x 128 rows (fp32)
 constexpr uint32_t kScBytes = 1024;            // s_x: 2 groups x 128 rows, s_w: 2 groups x 128 columns (fp16)
 constexpr uint32_t kEpiBoxBytes = 32 * 128;    // 32 rows x 64 bf16
-constexpr uint32_t kPairBytes = 2 * 128 * 4;   // per epilogue warp: two groups x 32 column pairs x 4 floats
 constexpr int kGroupBufs = 4;                  // TMEM: 4 x 128 fp32 columns
 
 __host__ __device__ constexpr uint32_t idesc_s8(int m, int n) {
@@ -89,6 +91,8 @@ struct SharedTail {
   uint64_t lr_empty;
   uint64_t sc_full[kScStages];
   uint64_t sc_empty[kScStages];
+  uint64_t cvt_full[kCvtStages];
+  uint64_t cvt_empty[kCvtStages];
   uint64_t grp_full[kGroupBufs];
   uint64_t grp_empty[kGroupBufs];
   uint32_t tmem_base;
@@ -96,7 +100,7 @@ struct SharedTail {
 };
 
 constexpr size_t kSmemBytes = 1024 + kStages * kStageBytes + kPkStages * kPkStageBytes + kLrBytes +
-                              kScStages * kScBytes + kEpiWarps * kEpiBoxBytes + kEpiWarps * kPairBytes +
+                              kScStages * kScBytes + kCvtStages * kCvtBytes + kEpiWarps * kEpiBoxBytes +
                               sizeof(SharedTail);
 static_assert(kSmemBytes <= 232448, "shared memory of one CTA");
 
@@ -118,9 +122,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* pk_smem = smem + kStages * kStageBytes;
   uint8_t* lr_smem = pk_smem + kPkStages * kPkStageBytes;
   uint8_t* sc_smem = lr_smem + kLrBytes;
-  uint8_t* epi_smem = sc_smem + kScStages * kScBytes;
-  float* pair_smem = reinterpret_cast<float*>(epi_smem + kEpiWarps * kEpiBoxBytes);
-  SharedTail* sh = reinterpret_cast<SharedTail*>(reinterpret_cast<uint8_t*>(pair_smem) + kEpiWarps * kPairBytes);
+  float* cvt_smem = reinterpret_cast<float*>(sc_smem + kScStages * kScBytes);
+  uint8_t* epi_smem = reinterpret_cast<uint8_t*>(cvt_smem) + kCvtStages * kCvtBytes;
+  SharedTail* sh = reinterpret_cast<SharedTail*>(epi_smem + kEpiWarps * kEpiBoxBytes);
   volatile int* abort_flag = &sh->abort_flag;
 
   const int warp = threadIdx.x >> 5;
@@ -143,7 +147,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     ptx::mbar_init(&sh->lr_empty, 1);
     for (int s = 0; s < kScStages; ++s) {
       ptx::mbar_init(&sh->sc_full[s], 1);
-      ptx::mbar_init(&sh->sc_empty[s], kEpiWarps);
+      ptx::mbar_init(&sh->sc_empty[s], kLoadWarps);
+    }
+    for (int s = 0; s < kCvtStages; ++s) {
+      ptx::mbar_init(&sh->cvt_full[s], kLoadWarps);
+      ptx::mbar_init(&sh->cvt_empty[s], kEpiWarps);
     }
     for (int b = 0; b < kGroupBufs; ++b) {
       ptx::mbar_init(&sh->grp_full[b], 1);
@@ -264,6 +272,29 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::fence_proxy_async_smem();        // generic-proxy writes -> visible to the tensor cores
         ptx::mbar_arrive(&sh->full[s]);
+        // the step's group scales as fp32 for the epilogue, once for all its warps: s_w / 256 of
+        // the 128 columns and s_x of the 128 rows, both groups (thread t: entries t + 64 u)
+        {
+          const int ss = it % kScStages, cs = it % kCvtStages;
+          if (!wait_bounded(&sh->sc_full[ss], (it / kScStages) & 1, abort_flag, p.err, kErrSiteGemmFull) ||
+              !wait_bounded(&sh->cvt_empty[cs], ((it / kCvtStages) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmEmpty)) {
+            ok = false;
+            break;
+          }
+          const __half* sch = reinterpret_cast<const __half*>(sc_smem + ss * kScBytes);   // s_x [2][128], s_w [2][128]
+          float* cv = cvt_smem + cs * (kCvtBytes / 4);                                    // s_w/256 [2][128], s_x [2][128]
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int e = threadIdx.x + 64 * u;
+            cv[e] = __half2float(sch[256 + e]) * 0.00390625f;
+            cv[256 + e] = __half2float(sch[e]);
+          }
+          __syncwarp();
+          if ((threadIdx.x & 31) == 0) {
+            ptx::mbar_arrive(&sh->sc_empty[ss]);
+            ptx::mbar_arrive(&sh->cvt_full[cs]);
+          }
+        }
       }
     }
   } else if (warp == kMmaWarp) {
@@ -304,7 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         __syncwarp();
       }
       if (!ok || nk_lr == 0) continue;
-      // low-rank branch: Z L2^T into one more group buffer (its first MMA overwrites the preset)
+      // low-rank branch: Z L2^T into one more group buffer (its first MMA overwrites it)
       const int b = gi % kGroupBufs;
       if (!wait_bounded(&sh->grp_empty[b], ((gi / kGroupBufs) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmAccEmpty)) {
         ok = false;
@@ -334,13 +365,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ epilogue (warps 4-11)
     // Each warp owns 32 rows (its TMEM lane quarter) x 64 columns and reads them in the
     // 16x256b shape: thread l holds rows {l/4, l/4 + 8} of each 16-row slab and the column
-    // pairs 8i + 2(l%4) + {0, 1}, i = 0..7, i.e. 4 rows x 16 columns.  A thread then needs
-    // the weight-scale pairs of 16 columns per group (8 shared loads) instead of 64.
+    // pairs 8i + 2(l%4) + {0, 1}, i = 0..7, i.e. 4 rows x 16 columns.  A thread then reads the
+    // weight scales of 16 columns per group (8 shared loads) instead of 64.
     const int e = warp - kEpiWarp0;
     const int q = warp & 3;                    // TMEM lane quarter (rows q*32 .. q*32+31)
     const int h = e >> 2;                      // 64-column half of the tile
     const int lr = lane >> 2, lc = lane & 3;   // row within an 8-row group, column pair within a chunk
-    float* pairs = pair_smem + e * (kPairBytes / 4);
     uint8_t* buf = epi_smem + e * kEpiBoxBytes;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 64;
     const int ngroups = G + (p.rank > 0 ? 1 : 0);
@@ -359,30 +389,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int b = gi % kGroupBufs;
         const uint32_t base = lane_base + b * kBN;
         float sa[4] = {1.f, 1.f, 1.f, 1.f};
-        const float* pr = pairs + (g & 1) * 128;
+        const float* cva = cvt_smem + ((sc_it + (g >> 1)) % kCvtStages) * (kCvtBytes / 4) + (g & 1) * 128;
         if (!lowrank) {
-          // this group's row scales and (s_w / 256, -B s_w / 256) for the warp's 64 columns
-          // (written by lane l for columns 2l, 2l + 1), prepared before the product is waited for
-          const int ss = (sc_it + (g >> 1)) % kScStages;
+          // this group's fp32 scales, converted once per K step by the widening warps
+          const int cs = (sc_it + (g >> 1)) % kCvtStages;
           if ((g & 1) == 0 &&
-              !wait_bounded(&sh->sc_full[ss], ((sc_it + (g >> 1)) / kScStages) & 1, abort_flag, p.err,
+              !wait_bounded(&sh->cvt_full[cs], ((sc_it + (g >> 1)) / kCvtStages) & 1, abort_flag, p.err,
                             kErrSiteGemmFull)) {
             ok = false;
             break;
           }
-          const uint8_t* sc = sc_smem + ss * kScBytes + (g & 1) * 256;
-          if (SVDQ_IN_SMEM(smem_raw, sc, 256, p.err) && SVDQ_IN_SMEM(smem_raw, sc + 512, 256, p.err) &&
-              SVDQ_IN_SMEM(smem_raw, pairs + (g & 1) * 128 + lane * 4, 16, p.err)) {
 #pragma unroll
-            for (int j = 0; j < 4; ++j)
-              sa[j] = __half2float(*reinterpret_cast<const __half*>(sc + (q * 32 + 8 * j + lr) * 2));
-            const float2 sw = __half22float2(*reinterpret_cast<const __half2*>(sc + 512 + (h * 64 + 2 * lane) * 2));
-            const float w0 = sw.x * 0.00390625f, w1 = sw.y * 0.00390625f;
-            *reinterpret_cast<float4*>(pairs + (g & 1) * 128 + lane * 4) =
-                make_float4(w0, w1, w0 * -kAccBiasF, w1 * -kAccBiasF);
-          }
-          __syncwarp();
-          if ((g & 1) == 1 && lane == 0) ptx::mbar_arrive(&sh->sc_empty[ss]);
+          for (int j = 0; j < 4; ++j) sa[j] = cva[256 + q * 32 + 8 * j + lr];
         }
         if (!wait_bounded(&sh->grp_full[b], (gi / kGroupBufs) & 1, abort_flag, p.err, kErrSiteGemmAccFull)) {
           ok = false;
@@ -406,10 +424,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         } else {
 #pragma unroll
           for (int i = 0; i < 8; ++i) {
-            const float4 s4 = SVDQ_IN_SMEM(smem_raw, pr + (4 * i + lc) * 4, 16, p.err)
-                                  ? *reinterpret_cast<const float4*>(pr + (4 * i + lc) * 4)
-                                  : make_float4(0.f, 0.f, 0.f, 0.f);
-            const float2 a2 = make_float2(s4.x, s4.y), b2 = make_float2(s4.z, s4.w);
+            const float* ap = cva + h * 64 + 8 * i + 2 * lc;
+            const float2 a2 = SVDQ_IN_SMEM(smem_raw, ap, 8, p.err) ? *reinterpret_cast<const float2*>(ap)
+                                                                   : make_float2(0.f, 0.f);
+            const float2 b2 = __fmul2_rn(a2, make_float2(-kAccBiasF, -kAccBiasF));   // -B s_w / 256, exact
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               // s32 256 D + the bits of B is the float B + 256 D exactly (|256 D| < 2^22)
@@ -419,6 +437,11 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc[j][i] = __ffma2_rn(tt, make_float2(sa[j], sa[j]), acc[j][i]);
             }
           }
+        }
+        if (!lowrank && (g & 1) == 1) {
+          // both groups of the K step have read their scales: the slot goes back
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&sh->cvt_empty[(sc_it + (g >> 1)) % kCvtStages]);
         }
       }
       sc_it += nk_main;
