@@ -24,7 +24,9 @@
 //     of the order of a hundred cycles on top of its bytes, so fewer, larger
 //     loads stream faster (when K is not a multiple of 256, two 2-D loads per
 //     operand and slot).  Every load lands in the issuing CTA's own shared
-//     memory and counts on the leader CTA's barrier (no multicast loads);
+//     memory and counts on the leader CTA's barrier (no multicast loads).  The
+//     operand and scale loads carry an L2 evict-last policy: every A and B tile
+//     is read by many clusters, while Y passes through L2 once;
 //   * the block scales (E4M3, one per 16 elements; 512-byte "128 rows x 4 groups"
 //     blocks) travel in a ring of their own whose slots also hold two main steps
 //     (one SFA and one SFB load per slot), loaded two main steps ahead of the
@@ -44,8 +46,9 @@
 //   * eight epilogue warps per CTA drain TMEM (tcgen05.ld) into registers and
 //     release the accumulator at once, then apply g_x g_w and the bias and store
 //     bf16 Y from registers while the next tile's MMAs run: each thread writes
-//     256 contiguous bytes of its row with 32-byte (one sector) stores, which
-//     halves the write requests of 16-byte stores (32 rows per warp instruction).
+//     256 contiguous bytes of its row with 32-byte (one sector) stores that do not
+//     allocate in L1, which halves the write requests of 16-byte stores (32 rows
+//     per warp instruction).
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cstdint>
@@ -189,6 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       int it = 0, mi = 0, si = 0;
       bool ok = true;
+      // A, B and their scales are re-read by the other clusters' tiles: evict them from L2
+      // after other lines (Y is written once and stored without allocating in L1)
+      const uint64_t keep = ptx::l2_evict_last_policy();
       // scale slot q = (tile j, steps 2u and 2u + 1) holds both steps' blocks: SFA [2 kSfBlk][512 B],
       // then SFB [2 row blocks][2 kSfBlk][512 B]; one TMA load per tensor and slot
       const int npair = (nk_main + 1) / 2;
@@ -206,8 +212,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t full_leader = ptx::mapa_shared(ptx::smem_u32(&sh->sf_full[ss]), 0);
           const uint32_t st = ptx::smem_u32(sf_smem + ss * kSfStageBytes);
           if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->sf_full[ss], kTxSf);
-          ptx::tma_load_3d_pair(st, &tmap_sfa, full_leader, 0, ks * kSfBlk, m0s / 128);
-          ptx::tma_load_3d_pair(st + 2 * kSfaBytes, &tmap_sfb, full_leader, 0, ks * kSfBlk, n0s / 128);
+          ptx::tma_load_3d_pair_hint(st, &tmap_sfa, full_leader, 0, ks * kSfBlk, m0s / 128, keep);
+          ptx::tma_load_3d_pair_hint(st + 2 * kSfaBytes, &tmap_sfb, full_leader, 0, ks * kSfBlk, n0s / 128, keep);
         }
       };
       for (int j = 0; j < tiles.count && ok; ++j) {
@@ -232,15 +238,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (p.op_pair) {
               // one load per operand: K steps k and k + 1 (a missing second step reads as zeros)
               if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], kTxMain);
-              ptx::tma_load_3d_pair(st, &tmap_a, full_leader, 0, m0, k);
-              ptx::tma_load_3d_pair(st + 2 * kABytes, &tmap_b, full_leader, 0, nb0, k);
+              ptx::tma_load_3d_pair_hint(st, &tmap_a, full_leader, 0, m0, k, keep);
+              ptx::tma_load_3d_pair_hint(st + 2 * kABytes, &tmap_b, full_leader, 0, nb0, k, keep);
             } else {
               if (rank == 0) ptx::mbar_arrive_expect_tx(&sh->full[s], two ? kTxMain : kTxMain / 2);
-              ptx::tma_load_2d_pair(st, &tmap_a, full_leader, k * (kKTile / 2), m0);
-              ptx::tma_load_2d_pair(st + 2 * kABytes, &tmap_b, full_leader, k * (kKTile / 2), nb0);
+              ptx::tma_load_2d_pair_hint(st, &tmap_a, full_leader, k * (kKTile / 2), m0, keep);
+              ptx::tma_load_2d_pair_hint(st + 2 * kABytes, &tmap_b, full_leader, k * (kKTile / 2), nb0, keep);
               if (two) {
-                ptx::tma_load_2d_pair(st + kABytes, &tmap_a, full_leader, (k + 1) * (kKTile / 2), m0);
-                ptx::tma_load_2d_pair(st + 3 * kABytes, &tmap_b, full_leader, (k + 1) * (kKTile / 2), nb0);
+                ptx::tma_load_2d_pair_hint(st + kABytes, &tmap_a, full_leader, (k + 1) * (kKTile / 2), m0, keep);
+                ptx::tma_load_2d_pair_hint(st + 3 * kABytes, &tmap_b, full_leader, (k + 1) * (kKTile / 2), nb0, keep);
               }
             }
             mi += two ? 2 : 1;
@@ -432,7 +438,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!in_n) {
         } else if (p.y_align32) {
-          ptx::st_global_v8(yrow + cl, o);
+          ptx::st_global_v8_na(yrow + cl, o);
         } else {
           *reinterpret_cast<uint4*>(yrow + cl) = make_uint4(o[0], o[1], o[2], o[3]);
           *reinterpret_cast<uint4*>(yrow + cl + 8) = make_uint4(o[4], o[5], o[6], o[7]);
