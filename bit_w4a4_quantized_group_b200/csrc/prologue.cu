@@ -17,7 +17,7 @@
 // warps that share a row strip are summed in a fixed order (deterministic).
 //
 // Few rows (small batches) leave most SMs idle, since a CTA owns 32 rows over all of K.  The
-// 4-bit formats then split each row block's K stages over a cluster of up to 4 CTAs: codes
+// 4-bit formats then split each row block's K stages over a cluster of up to 8 CTAs: codes
 // and scales are local to their groups, and the Z partials of the CTAs are added by CTA 0
 // of the cluster through distributed shared memory, in CTA order (deterministic).
 //
@@ -634,14 +634,49 @@ int stages_for() {
   return s;
 }
 
+// Largest number of clusters of `ks` split CTAs that can be resident at once (0 if none or
+// on error), queried once per template instance, split size and shared-memory size.
+template <int FMT, int RANK>
+static int resident_clusters(int ks, size_t smem) {
+  static int cached[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
+  static size_t cached_smem[9] = {};
+  if (ks < 2 || ks > 8) return 0;
+  if (cached[ks] >= 0 && cached_smem[ks] == smem) return cached[ks];
+  auto kern = prologue_kernel<FMT, RANK, true>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ks), 1, 1);
+  cfg.blockDim = dim3(32 * (compute_warps(RANK) + 1), 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached_smem[ks] = smem;
+  cached[ks] = n;
+  return n;
+}
+
 template <int FMT, int RANK>
 static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, ProParams p, cudaStream_t stream) {
   p.stages = stages_for<FMT, RANK>();
   if (p.stages < 2) return cudaErrorInvalidConfiguration;
   const size_t smem = smem_bytes_for<FMT, RANK>(p.stages);
   const int blocks = p.Mpad / kProRows;
-  // K split for small batches (4-bit formats): the largest cluster of up to 4 CTAs per row
-  // block that keeps one wave on the SMs and leaves no CTA without a stage.
+  // K split for small batches (4-bit formats): the largest cluster of up to 8 CTAs per row
+  // block that keeps one wave on the SMs (every cluster resident at once) and leaves no CTA
+  // without a stage.
   constexpr int BK = 64 * (compute_warps(RANK) / 2);
   const int nkt_all = (p.K + BK - 1) / BK;
   int sms = 0, dev = 0;
@@ -649,9 +684,10 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
     return cudaErrorInvalidDevice;
   p.ksplit = 1;
   if (FMT != kFmtW8a8) {
-    for (int ks = 4; ks >= 2; --ks) {
+    for (int ks = 8; ks >= 2; --ks) {
       const int nks = (nkt_all + ks - 1) / ks;
-      if (ks <= nkt_all && nks * (ks - 1) < nkt_all && blocks * ks <= sms) {
+      if (ks <= nkt_all && nks * (ks - 1) < nkt_all && blocks * ks <= sms &&
+          resident_clusters<FMT, RANK>(ks, smem) >= blocks) {
         p.ksplit = ks;
         break;
       }

@@ -66,7 +66,7 @@ def _check_prologue(fmt, X, lam, gx, L1_rk):
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,K,rank", [(300, 640, 32), (128, 256, 16), (1, 128, 0), (257, 1024, 48),
                                       (96, 512, 128), (256, 3072, 32), (100, 2048, 16), (64, 1280, 128),
-                                      (64, 2048, 0), (200, 3072, 0)])
+                                      (64, 2048, 0), (200, 3072, 0), (64, 3584, 16), (256, 12288, 32)])
 def test_prologue_parity(fmt, M, K, rank):
     layer, prep = _layer(M, K, 256, rank, seed=7 + M + rank, fmt=fmt)
     _check_prologue(fmt, layer.X, prep["lam"], prep["act_gscale"], prep["L1_rk"] if rank else None)
@@ -446,7 +446,8 @@ def test_layer_random_shapes(case):
 
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
-@pytest.mark.parametrize("M,K,N,rank", [(256, 3072, 3072, 32), (1024, 3072, 1024, 64), (40, 2048, 512, 16)])
+@pytest.mark.parametrize("M,K,N,rank", [(256, 3072, 3072, 32), (1024, 3072, 1024, 64), (40, 2048, 512, 16),
+                                        (256, 12288, 512, 32)])
 def test_layer_small_batch_k_split(fmt, M, K, N, rank):
     """Small batches, where the prologue splits each row block's K stages over a cluster of
     CTAs and adds their Z partials through distributed shared memory; the whole layer
