@@ -171,6 +171,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
+  // the set-up above may overlap the end of the prologue kernel; its outputs (A codes and
+  // scales, Z) are read only after it has completed
+  ptx::griddep_wait();
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ TMA producer
@@ -496,7 +499,18 @@ cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const
                                        static_cast<int>(smem));
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
-  gemm_int4_kernel<<<grid, kThreads, smem, s>>>(ta, tb, tz, tl2, ty, tsa, tsb, p);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start under the prologue
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  e = cudaLaunchKernelEx(&cfg, gemm_int4_kernel, ta, tb, tz, tl2, ty, tsa, tsb, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
 

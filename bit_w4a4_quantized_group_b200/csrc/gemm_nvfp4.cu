@@ -176,6 +176,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   ptx::cluster_sync();
   ptx::tc_fence_after();
   const uint32_t tmem = sh->tmem_base;
+  // the set-up above may overlap the end of the prologue kernel; its outputs (A codes and
+  // scales, Z) are read only after it has completed
+  ptx::griddep_wait();
 
   if (warp == kProdWarp) {
     // ------------------------------------------------------------ producer (both CTAs)
@@ -508,13 +511,15 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorM
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start under the prologue
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   e = cudaLaunchKernelEx(&cfg, gemm_fp4_kernel<MX>, ta, tb, tsfa, tsfb, tz, tl2, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();

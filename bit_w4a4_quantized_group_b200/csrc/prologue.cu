@@ -166,6 +166,9 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  // the GEMM launched after this kernel may start its own set-up now (on SMs this grid leaves
+  // free); it reads this kernel's outputs only after the whole grid has completed
+  ptx::griddep_launch_dependents();
 
   if (warp == NW) {
     // ---------------------------------------------------------------- producer warp

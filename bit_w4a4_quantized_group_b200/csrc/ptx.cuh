@@ -277,6 +277,14 @@ __device__ __forceinline__ void tma_load_2d_pair(uint32_t dst, const CUtensorMap
       "l"(reinterpret_cast<uint64_t>(map)), "r"(bar_cluster), "r"(x), "r"(y)
       : "memory");
 }
+// Programmatic dependent launch: a grid lets the next kernel on its stream start once every
+// CTA has issued launch_dependents (or exited); the next kernel's griddepcontrol.wait returns
+// only when this grid has completed and its memory writes are visible.  Without the launch
+// attribute that allows the overlap, the wait returns at once.
+__device__ __forceinline__ void griddep_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void griddep_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 // L2 policy for operand tiles that other CTAs re-read: evict them after other lines
 __device__ __forceinline__ uint64_t l2_evict_last_policy() {
   uint64_t pol;

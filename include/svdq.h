@@ -181,6 +181,9 @@ svdq_status svdq_quantize_act_lowrank_down(svdq_format fmt, int64_t M, int64_t K
  * an s32 accumulator and the low-rank product in a second, fp32 accumulator, both on
  * the tensor cores and combined in the epilogue (act_gscale = w_gscale = 1, L2s = L2).
  * Z and L2s may be NULL when rank == 0; bias may be NULL.
+ * Stream order is kept: the GEMM is launched so that it may start its set-up while the
+ * kernel before it on the stream (normally this library's prologue) finishes, but it reads
+ * its inputs only after that kernel has completed (programmatic dependent launch).
  */
 svdq_status svdq_w4a4_gemm_lowrank_up(svdq_format fmt, int64_t M, int64_t N, int64_t K, int rank,
                                       const void* a_codes, const void* a_scales, float act_gscale,
