@@ -165,18 +165,20 @@ def pack_weight_np(fmt, R_nk, L1_rk, L2_nr, act_gscale: float = 1.0):
             "L1_bf16": l1b[: rank * K].reshape(rank, K), "L2_bf16": l2b[: N * rank].reshape(N, rank)}
 
 
-def quantize_act_lowrank_down_t(fmt, X, lam, act_gscale, L1, a_codes, a_scales, Z):
-    """Device prologue on torch tensors (X [M, K] bf16, L1 [r, K] bf16 viewed as any 2-byte dtype)."""
+def quantize_act_lowrank_down_t(fmt, X, lam, act_gscale, L1, a_codes, a_scales, Z, stream=None):
+    """Device prologue on torch tensors (X [M, K] bf16, L1 [r, K] bf16 viewed as any 2-byte dtype).
+    `stream` is a raw cudaStream_t handle; None means torch's current stream."""
     M, K = X.shape
     rank = 0 if L1 is None else L1.shape[0]
     st = svdq_quantize_act_lowrank_down(fmt, M, K, rank, _ptr(X), _ptr(lam), act_gscale, _ptr(L1),
-                                        _ptr(a_codes), _ptr(a_scales), _ptr(Z), _stream())
+                                        _ptr(a_codes), _ptr(a_scales), _ptr(Z),
+                                        _stream() if stream is None else stream)
     _check(st, "svdq_quantize_act_lowrank_down")
 
 
 def w4a4_gemm_lowrank_up_t(fmt, M, N, K, rank, a_codes, a_scales, act_gscale, w_codes, w_scales, w_gscale,
-                           Z, L2, bias, Y):
+                           Z, L2, bias, Y, stream=None):
     st = svdq_w4a4_gemm_lowrank_up(fmt, M, N, K, rank, _ptr(a_codes), _ptr(a_scales), act_gscale,
                                    _ptr(w_codes), _ptr(w_scales), w_gscale, _ptr(Z), _ptr(L2), _ptr(bias),
-                                   _ptr(Y), _stream())
+                                   _ptr(Y), _stream() if stream is None else stream)
     _check(st, "svdq_w4a4_gemm_lowrank_up")

@@ -495,8 +495,7 @@ cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const
                              const CUtensorMap& tsb, const GemmParams& p, int num_sms,
                              cudaStream_t s) {
   const size_t smem = gemm_int4_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_int4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(gemm_int4_kernel), smem);
   if (e != cudaSuccess) return e;
   const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
   cudaLaunchConfig_t cfg = {};

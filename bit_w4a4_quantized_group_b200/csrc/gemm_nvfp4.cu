@@ -500,8 +500,7 @@ cudaError_t launch(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorM
                    const CUtensorMap& tz, const CUtensorMap& tl2, const GemmParams& p,
                    int num_sms, cudaStream_t s) {
   const size_t smem = smem_bytes<MX>();
-  cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<MX>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(gemm_fp4_kernel<MX>), smem);
   if (e != cudaSuccess) return e;
   int clusters = max_active_clusters<MX>(smem);
   if (clusters <= 0) clusters = num_sms / 2;

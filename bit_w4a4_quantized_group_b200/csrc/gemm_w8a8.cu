@@ -392,8 +392,7 @@ cudaError_t launch_gemm_w8a8(const CUtensorMap& ta, const CUtensorMap& tb, const
                              const CUtensorMap& tl2, const CUtensorMap& ty, const GemmParams& p, int num_sms,
                              cudaStream_t s) {
   const size_t smem = smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(gemm_w8a8_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(gemm_w8a8_kernel), smem);
   if (e != cudaSuccess) return e;
   int clusters = max_active_clusters(smem);
   if (clusters <= 0) clusters = num_sms / 2;

@@ -646,7 +646,7 @@ static int resident_clusters(int ks, size_t smem) {
   if (ks < 2 || ks > 8) return 0;
   if (cached[ks] >= 0 && cached_smem[ks] == smem) return cached[ks];
   auto kern = prologue_kernel<FMT, RANK, true>;
-  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem)) != cudaSuccess) {
+  if (set_smem_limit_once(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -698,13 +698,13 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
   }
   if (p.ksplit == 1) {
     auto kern = prologue_kernel<FMT, RANK, false>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
     if (e != cudaSuccess) return e;
     kern<<<blocks, 32 * (compute_warps(RANK) + 1), smem, stream>>>(tx, tl1, p);
     return cudaGetLastError();
   }
   auto kern = prologue_kernel<FMT, RANK, true>;
-  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(kern), smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(blocks * p.ksplit, 1, 1);

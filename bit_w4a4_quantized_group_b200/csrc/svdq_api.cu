@@ -78,6 +78,34 @@ bool make_tmap_sf(CUtensorMap* m, const void* base, int64_t rows_pad, int64_t K,
                       kblocks * 512, 64, static_cast<uint32_t>(2 * 256 / (4 * g)), blocks);
 }
 
+}  // namespace
+
+cudaError_t set_smem_limit_once(const void* kernel, size_t smem) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  struct Seen {
+    const void* kernel;
+    int dev;
+    size_t smem;
+  };
+  static Seen seen[512];
+  static int n = 0;
+  static std::mutex mu;
+  {
+    std::lock_guard<std::mutex> lock(mu);
+    for (int i = 0; i < n; ++i)
+      if (seen[i].kernel == kernel && seen[i].dev == dev && seen[i].smem == smem) return cudaSuccess;
+  }
+  e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  std::lock_guard<std::mutex> lock(mu);
+  if (n < 512) seen[n++] = Seen{kernel, dev, smem};
+  return cudaSuccess;
+}
+
+namespace {
+
 int device_sm_count() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;

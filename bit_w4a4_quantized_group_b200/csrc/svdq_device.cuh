@@ -112,6 +112,10 @@ constexpr int kProBoxes = 4;   // 64-column boxes per prologue TMA load
 
 // Self-test of the bounded wait: a wait on a barrier nothing arrives at.
 cudaError_t launch_selftest_bounded_wait(int* err, uint64_t limit_ns, cudaStream_t s);
+// Raises a kernel's dynamic shared-memory limit to `smem` bytes on the current device, once
+// per (kernel, device, size): the attribute belongs to the function in the device's context,
+// and setting it on every launch costs host time.
+cudaError_t set_smem_limit_once(const void* kernel, size_t smem);
 
 struct ProParams {
   int M, K, rank, Mpad, stages;

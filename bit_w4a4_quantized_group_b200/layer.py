@@ -73,11 +73,12 @@ class W4A4LowRankLinear:
         ws = self.workspace(M)
         if Y is None:
             Y = torch.empty((M, self.N), dtype=torch.bfloat16, device=self.device)
+        stream = torch.cuda.current_stream(self.device).cuda_stream     # one lookup for both calls
         B.quantize_act_lowrank_down_t(self.fmt, X, self.lam, self.act_gscale, self.L1,
-                                      ws["a_codes"], ws["a_scales"], ws["Z"])
+                                      ws["a_codes"], ws["a_scales"], ws["Z"], stream)
         B.w4a4_gemm_lowrank_up_t(self.fmt, M, self.N, K, self.rank, ws["a_codes"], ws["a_scales"],
                                  self.act_gscale, self.w_codes, self.w_scales, self.w_gscale,
-                                 ws["Z"], self.L2, self.bias, Y)
+                                 ws["Z"], self.L2, self.bias, Y, stream)
         if check:
             st, site = B.svdq_get_last_device_error(torch.cuda.current_stream(self.device).cuda_stream)
             if st != B.SVDQ_OK:
