@@ -1,4 +1,5 @@
-"""The layer's forward (prologue + GEMM, two C-ABI calls) captured into a CUDA graph.
+"""The layer's forward (prologue + GEMM, two C-ABI calls) in a CUDA graph and in interleaved
+streams of calls.
 
 A captured forward replays the same two launches with the same tensor maps, so a replay
 on new inputs written into the captured input buffer must give the eager call's output
@@ -55,3 +56,33 @@ def test_forward_replays_from_a_cuda_graph(fmt, M, K, N, rank):
     st, site = B.svdq_get_last_device_error(None)
     assert st == B.SVDQ_OK, (st, site)
     del g
+
+
+@pytest.mark.gpu
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "w8a8"])
+def test_interleaved_calls_of_two_layers_keep_stream_order(fmt):
+    """Prologue A, prologue B, GEMM A, GEMM B on one stream.  Each GEMM may start its set-up
+    under the kernel just before it (here the other layer's prologue) and must still read
+    its own, completed prologue outputs: Y equals the plain sequential calls bit for bit."""
+    from bit_w4a4_quantized_group_b200 import binding as B
+    dev = torch.device("cuda", 0)
+    la = _layer(fmt, 512, 2048, 1024, 32, seed=11)
+    lb = _layer(fmt, 256, 2048, 1024, 16, seed=12)
+    gen = torch.Generator(device=dev).manual_seed(5)
+    Xa = (torch.randn(512, 2048, device=dev, generator=gen) * 2).to(torch.bfloat16)
+    Xb = (torch.randn(256, 2048, device=dev, generator=gen) * 2).to(torch.bfloat16)
+    Ya_ref = la.forward(Xa)
+    Yb_ref = lb.forward(Xb)
+    torch.cuda.synchronize()
+    Ya = torch.empty_like(Ya_ref)
+    Yb = torch.empty_like(Yb_ref)
+    for _ in range(3):
+        la.prologue_only(Xa)
+        lb.prologue_only(Xb)
+        la.gemm_only(512, Ya)
+        lb.gemm_only(256, Yb)
+    torch.cuda.synchronize()
+    assert torch.equal(Ya.view(torch.int16), Ya_ref.view(torch.int16))
+    assert torch.equal(Yb.view(torch.int16), Yb_ref.view(torch.int16))
+    st, site = B.svdq_get_last_device_error(None)
+    assert st == B.SVDQ_OK, (st, site)
