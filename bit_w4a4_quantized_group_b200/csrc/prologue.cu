@@ -637,14 +637,17 @@ int stages_for() {
   return s;
 }
 
-// Largest number of clusters of `ks` split CTAs that can be resident at once (0 if none or
-// on error), queried once per template instance, split size and shared-memory size.
+// Largest number of clusters of `ks` split CTAs that can be resident at once on the current
+// device (0 if none or on error), queried once per device, template instance, split size and
+// shared-memory size.
 template <int FMT, int RANK>
 static int resident_clusters(int ks, size_t smem) {
-  static int cached[9] = {-1, -1, -1, -1, -1, -1, -1, -1, -1};
-  static size_t cached_smem[9] = {};
-  if (ks < 2 || ks > 8) return 0;
-  if (cached[ks] >= 0 && cached_smem[ks] == smem) return cached[ks];
+  constexpr int kDevs = 64;
+  static int cached[kDevs][9];            // 0: not queried yet, else 1 + the figure
+  static size_t cached_smem[kDevs][9];
+  int dev = 0;
+  if (ks < 2 || ks > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return 0;
+  if (cached[dev][ks] > 0 && cached_smem[dev][ks] == smem) return cached[dev][ks] - 1;
   auto kern = prologue_kernel<FMT, RANK, true>;
   if (set_smem_limit_once(reinterpret_cast<const void*>(kern), smem) != cudaSuccess) {
     cudaGetLastError();
@@ -666,8 +669,8 @@ static int resident_clusters(int ks, size_t smem) {
     cudaGetLastError();
     n = 0;
   }
-  cached_smem[ks] = smem;
-  cached[ks] = n;
+  cached_smem[dev][ks] = smem;
+  cached[dev][ks] = n + 1;
   return n;
 }
 
