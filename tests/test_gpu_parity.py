@@ -172,7 +172,8 @@ def _gemm_case(fmt, M, N, K, rank, seed, with_bias=True, y_offset=0):
 
 @pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,N,K,rank", [(300, 640, 640, 32), (256, 512, 512, 16), (128, 256, 256, 0),
-                                        (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64)])
+                                        (200, 384, 384, 48), (129, 256, 1024, 128), (64, 768, 256, 64),
+                                        (130, 256, 128, 16), (1, 128, 128, 0), (257, 128, 384, 32)])
 def test_gemm_parity(fmt, M, N, K, rank):
     _gemm_case(fmt, M, N, K, rank, seed=11 + M + N + rank)
 
