@@ -563,23 +563,25 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
         zb[(g + 8) * RANK + c + 1] = acc[nt][3];
       }
       named_barrier_sync(1, 32 * NW);
-      // the two warps of phase 0 sum the partials in phase order and store bf16
-      if (phase == 0) {
+      // all compute warps sum the partials of the CTA's 32 x RANK outputs, two columns per
+      // thread, each in phase order, and store bf16 (or this CTA's partial for the K split)
+      {
         constexpr int R1 = RANK > 0 ? RANK : 1;
-        for (int idx = lane; idx < 16 * R1 / 2; idx += 32) {
-          const int r = (idx * 2) / R1, c = (idx * 2) % R1;
+        for (int idx = warp * 32 + lane; idx < 16 * R1; idx += 32 * NW) {
+          const int sr = (idx * 2) / R1, c = (idx * 2) % R1;   // row of the 32-row block, column
+          const int st = sr >> 4, r = sr & 15;
           float s0 = 0.f, s1 = 0.f;
 #pragma unroll
           for (int ph = 0; ph < BOXES; ++ph) {
-            const float* src = zbuf + ((ph * 2 + strip) * 16 + r) * R1 + c;
+            const float* src = zbuf + ((ph * 2 + st) * 16 + r) * R1 + c;
             s0 += src[0];
             s1 += src[1];
           }
-          const int row = m0 + strip * 16 + r;
+          const int row = m0 + sr;
           if (SPLIT) {
             float* zsum = zbuf + BOXES * 2 * 16 * R1;         // this CTA's partial [32][RANK]
-            zsum[(strip * 16 + r) * R1 + c] = s0;
-            zsum[(strip * 16 + r) * R1 + c + 1] = s1;
+            zsum[sr * R1 + c] = s0;
+            zsum[sr * R1 + c + 1] = s1;
           } else if (row < p.M) {
             __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
             *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * R1 + c) = v;
@@ -595,20 +597,35 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   if (RANK > 0 && SPLIT) {
     constexpr int R1 = RANK > 0 ? RANK : 1;
     ptx::cluster_sync();                                      // every partial is in shared memory
-    if (split == 0 && warp < 2) {
-      const int strip = warp;                                 // warps 0 and 1: phase 0, both strips
+    if (split == 0) {
+      // every thread of CTA 0 takes two columns of the 32 x RANK block: the peers' partials
+      // are all requested before any is added (remote reads overlap), then added in CTA order
+      constexpr int kMaxSplit = 8;
       const float* zsum = reinterpret_cast<const float*>(smem) + BOXES * 2 * 16 * R1;
       const uint32_t zaddr = ptx::smem_u32(zsum);
-      for (int idx = lane; idx < 16 * R1 / 2; idx += 32) {
-        const int r = (idx * 2) / R1, c = (idx * 2) % R1;
-        const int o = (strip * 16 + r) * R1 + c;
-        float s0 = zsum[o], s1 = zsum[o + 1];
-        for (int q = 1; q < p.ksplit; ++q) {
-          const uint32_t a = ptx::mapa_shared(zaddr + static_cast<uint32_t>(o) * 4u, static_cast<uint32_t>(q));
-          s0 += ptx::ld_shared_cluster_f32(a);
-          s1 += ptx::ld_shared_cluster_f32(a + 4u);
+      for (int idx = threadIdx.x; idx < 16 * R1; idx += blockDim.x) {
+        const int sr = (idx * 2) / R1, c = (idx * 2) % R1;
+        const int o = sr * R1 + c;
+        float v0[kMaxSplit - 1], v1[kMaxSplit - 1];
+#pragma unroll
+        for (int q = 1; q < kMaxSplit; ++q) {
+          v0[q - 1] = 0.f;
+          v1[q - 1] = 0.f;
+          if (q < p.ksplit) {
+            const uint32_t a = ptx::mapa_shared(zaddr + static_cast<uint32_t>(o) * 4u, static_cast<uint32_t>(q));
+            v0[q - 1] = ptx::ld_shared_cluster_f32(a);
+            v1[q - 1] = ptx::ld_shared_cluster_f32(a + 4u);
+          }
         }
-        const int row = m0 + strip * 16 + r;
+        float s0 = zsum[o], s1 = zsum[o + 1];
+#pragma unroll
+        for (int q = 1; q < kMaxSplit; ++q) {
+          if (q < p.ksplit) {
+            s0 += v0[q - 1];
+            s1 += v1[q - 1];
+          }
+        }
+        const int row = m0 + sr;
         if (row < p.M) {
           __nv_bfloat162 v = __floats2bfloat162_rn(s0, s1);
           *reinterpret_cast<__nv_bfloat162*>(p.Z + static_cast<size_t>(row) * R1 + c) = v;
