@@ -112,6 +112,7 @@ __device__ __forceinline__ uint2 int4x8_to_s8x8_x16(uint32_t w) {
 
 __device__ __forceinline__ float2 u2f2(uint32_t a, uint32_t b) { return make_float2(__uint_as_float(a), __uint_as_float(b)); }
 
+template <bool SPLIT>
 __global__ void __launch_bounds__(kThreads, 1)
     gemm_int4_kernel(const __grid_constant__ CUtensorMap tmap_a, const __grid_constant__ CUtensorMap tmap_b,
                      const __grid_constant__ CUtensorMap tmap_z, const __grid_constant__ CUtensorMap tmap_l2,
@@ -130,9 +131,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int K = p.K;
-  const int G = K / 64;
   const int nk_main = (K + kKStep - 1) / kKStep;
-  const int nk_lr = (p.rank + 63) / 64;
+  // K split (few tiles): the S CTAs of a cluster share one tile, CTA q taking the K steps
+  // [kb, ke) and CTA 0 also the low-rank group; without the split a CTA runs whole tiles.
+  const int S = SPLIT ? p.ksplit : 1;
+  const int sq = SPLIT ? static_cast<int>(ptx::cluster_ctarank()) : 0;
+  const int t_first = SPLIT ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
+  const int t_step = SPLIT ? static_cast<int>(gridDim.x) / S : static_cast<int>(gridDim.x);
+  const int nks = (nk_main + S - 1) / S;
+  const int kb = SPLIT ? min(nk_main, sq * nks) : 0;
+  const int ke = SPLIT ? min(nk_main, kb + nks) : nk_main;
+  const int nk_lr = sq == 0 ? (p.rank + 63) / 64 : 0;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -182,9 +191,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::prefetch_tmap(&tmap_b);
       int pi = 0, li = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+      for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
         const int m0 = (t % p.tiles_m) * kBM, n0 = (t / p.tiles_m) * kBN;
-        for (int k = 0; k < nk_main; ++k, ++pi) {
+        for (int k = kb; k < ke; ++k, ++pi) {
           const int s = pi % kPkStages;
           if (!wait_bounded(&sh->pk_empty[s], ((pi / kPkStages) & 1) ^ 1u, abort_flag, p.err, kErrSiteGemmEmpty)) {
             ok = false;
@@ -221,8 +230,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------ widening warps
     int it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-      for (int k = 0; k < nk_main; ++k, ++it) {
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
+      for (int k = kb; k < ke; ++k, ++it) {
         const int ps = it % kPkStages;
         const int s = it % kStages;
         if (!wait_bounded(&sh->pk_full[ps], (it / kPkStages) & 1, abort_flag, p.err, kErrSiteGemmConvFull)) {
@@ -306,8 +315,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = true;
     const uint32_t id8 = idesc_s8(kBM, kBN);
     const uint32_t id16 = idesc_bf16(kBM, kBN);
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
-      for (int k = 0; k < nk_main && ok; ++k, ++it) {
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
+      for (int k = kb; k < ke && ok; ++k, ++it) {
         const int s = it % kStages;
         if (!wait_bounded(&sh->full[s], (it / kStages) & 1, abort_flag, p.err, kErrSiteGemmConvFull)) {
           ok = false;
@@ -376,10 +385,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int lr = lane >> 2, lc = lane & 3;   // row within an 8-row group, column pair within a chunk
     uint8_t* buf = epi_smem + e * kEpiBoxBytes;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(q * 32) << 16) + h * 64;
-    const int ngroups = G + (p.rank > 0 ? 1 : 0);
+    const int gm = 2 * (ke - kb);              // this CTA's groups of the 4-bit product
+    const int ngroups = gm + (nk_lr > 0 ? 1 : 0);
     int gi = 0, sc_it = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < p.num_tiles && ok; t += gridDim.x) {
+    for (int t = t_first; t < p.num_tiles && ok; t += t_step) {
       const int m0 = (t % p.tiles_m) * kBM, n0 = (t / p.tiles_m) * kBN;
       const int col0 = n0 + h * 64;
       float2 acc[4][8];                        // [row j = 2 slab + half][chunk i]
@@ -388,7 +398,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < 8; ++i) acc[j][i] = make_float2(0.f, 0.f);
       for (int g = 0; g < ngroups; ++g, ++gi) {
-        const bool lowrank = g == G;
+        const bool lowrank = g == gm;
         const int b = gi % kGroupBufs;
         const uint32_t base = lane_base + b * kBN;
         float sa[4] = {1.f, 1.f, 1.f, 1.f};
@@ -447,8 +457,23 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (lane == 0) ptx::mbar_arrive(&sh->cvt_empty[(sc_it + (g >> 1)) % kCvtStages]);
         }
       }
-      sc_it += nk_main;
+      sc_it += ke - kb;
       if (!ok) break;
+      if (SPLIT) {
+        // this CTA's fp32 partial of the tile to shared memory (the int8 ring is idle now: the
+        // last group's MMAs have completed), float4 k of thread x at [k][thread]
+        float4* part = reinterpret_cast<float4*>(smem);
+        const int x = e * 32 + lane;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int i = 0; i < 8; i += 2) {
+            float4* dst = part + ((j * 4 + i / 2) * (kEpiWarps * 32) + x);
+            if (SVDQ_IN_SMEM(smem_raw, dst, 16, p.err))
+              *dst = make_float4(acc[j][i].x, acc[j][i].y, acc[j][i + 1].x, acc[j][i + 1].y);
+          }
+        continue;
+      }
       // Y = acc + bias -> bf16, one 32-row x 64-column 128B-swizzled box and a TMA store
       if (lane == 0) ptx::bulk_wait_group_read<0>();
       __syncwarp();
@@ -478,6 +503,56 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   }
 
+  if (SPLIT) {
+    // CTA 0 adds the partials of the cluster's CTAs in CTA order (its own first), then the bias,
+    // and writes Y.  Every thread of every CTA reaches both cluster barriers, also after a wait
+    // that ran out above (the outputs are then undefined and the error word says so).
+    ptx::cluster_sync();                                  // every partial is in shared memory
+    if (sq == 0 && warp >= kEpiWarp0 && t_first < p.num_tiles) {
+      const int e = warp - kEpiWarp0, q = warp & 3, h = e >> 2, lr = lane >> 2, lc = lane & 3;
+      const int m0 = (t_first % p.tiles_m) * kBM, n0 = (t_first / p.tiles_m) * kBN;
+      const int col0 = n0 + h * 64;
+      const int x = e * 32 + lane;
+      const float4* part = reinterpret_cast<const float4*>(smem);
+      float4 sum[16];
+#pragma unroll
+      for (int k = 0; k < 16; ++k) sum[k] = part[k * (kEpiWarps * 32) + x];
+      const uint32_t pbase = ptx::smem_u32(smem);
+      for (int r = 1; r < S; ++r) {
+        float4 v[16];
+#pragma unroll
+        for (int k = 0; k < 16; ++k)                      // all of a peer's values in flight at once
+          v[k] = ptx::ld_shared_cluster_v4f32(
+              ptx::mapa_shared(pbase + static_cast<uint32_t>((k * (kEpiWarps * 32) + x) * 16), static_cast<uint32_t>(r)));
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          sum[k].x += v[k].x;
+          sum[k].y += v[k].y;
+          sum[k].z += v[k].z;
+          sum[k].w += v[k].w;
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        float2 bv = make_float2(0.f, 0.f);
+        const int c = col0 + 8 * i + 2 * lc;
+        if (p.bias && SVDQ_IN_GLOBAL(c + 2 <= p.N, p.err)) {
+          const uint32_t bw = __ldg(reinterpret_cast<const unsigned int*>(p.bias + c));
+          bv = make_float2(__uint_as_float(bw << 16), __uint_as_float(bw & 0xFFFF0000u));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float4 f = sum[j * 4 + i / 2];
+          const float2 a = (i & 1) ? make_float2(f.z, f.w) : make_float2(f.x, f.y);
+          const int row = m0 + q * 32 + 8 * j + lr;
+          if (row < p.M && SVDQ_IN_GLOBAL(c + 2 <= p.N, p.err))
+            *reinterpret_cast<__nv_bfloat162*>(p.Y + static_cast<size_t>(row) * p.N + c) =
+                __floats2bfloat162_rn(a.x + bv.x, a.y + bv.y);
+        }
+      }
+    }
+    ptx::cluster_sync();                                  // peers keep their partials until read
+  }
   ptx::tc_fence_before();
   __syncthreads();
   if (warp == kMmaWarp) {
@@ -490,25 +565,85 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 size_t gemm_int4_smem_bytes() { return kSmemBytes; }
 
+namespace {
+
+// Largest number of clusters of `ks` CTAs of the split kernel that can be resident at once on
+// the current device (0 if none or on error), queried once per device and split size.
+int int4_resident_clusters(int ks, size_t smem) {
+  constexpr int kDevs = 64;
+  static int cached[kDevs][9];            // 0: not queried yet, else 1 + the figure
+  int dev = 0;
+  if (ks < 2 || ks > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kDevs) return 0;
+  if (cached[dev][ks] > 0) return cached[dev][ks] - 1;
+  if (set_smem_limit_once(reinterpret_cast<const void*>(gemm_int4_kernel<true>), smem) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(ks), 1, 1);
+  cfg.blockDim = dim3(kThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(ks);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, gemm_int4_kernel<true>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    n = 0;
+  }
+  cached[dev][ks] = n + 1;
+  return n;
+}
+
+}  // namespace
+
 cudaError_t launch_gemm_int4(const CUtensorMap& ta, const CUtensorMap& tb, const CUtensorMap& tz,
                              const CUtensorMap& tl2, const CUtensorMap& ty, const CUtensorMap& tsa,
                              const CUtensorMap& tsb, const GemmParams& p, int num_sms,
                              cudaStream_t s) {
   const size_t smem = gemm_int4_smem_bytes();
-  cudaError_t e = set_smem_limit_once(reinterpret_cast<const void*>(gemm_int4_kernel), smem);
+  // Few tiles (small batches) leave most SMs idle, and each tile runs its K groups one after
+  // another at the epilogue's pace: split each tile's K steps over a cluster of up to 8 CTAs
+  // (the largest split that leaves every CTA a step and keeps all clusters resident at once).
+  GemmParams q = p;
+  q.ksplit = 1;
+  const int nk_main = p.K / kKStep;
+  if (p.num_tiles * 2 <= num_sms) {
+    for (int ks = 8; ks >= 2; --ks) {
+      const int nks = (nk_main + ks - 1) / ks;
+      if (ks <= nk_main && nks * (ks - 1) < nk_main && p.num_tiles * ks <= num_sms &&
+          int4_resident_clusters(ks, smem) >= p.num_tiles) {
+        q.ksplit = ks;
+        break;
+      }
+    }
+  }
+  const bool split = q.ksplit > 1;
+  const void* kern = split ? reinterpret_cast<const void*>(gemm_int4_kernel<true>)
+                           : reinterpret_cast<const void*>(gemm_int4_kernel<false>);
+  cudaError_t e = set_smem_limit_once(kern, smem);
   if (e != cudaSuccess) return e;
-  const int grid = p.num_tiles < num_sms ? p.num_tiles : num_sms;
+  const int grid = split ? p.num_tiles * q.ksplit : (p.num_tiles < num_sms ? p.num_tiles : num_sms);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid), 1, 1);
   cfg.blockDim = dim3(kThreads, 1, 1);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // may start under the prologue
   attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = static_cast<unsigned>(q.ksplit);
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  e = cudaLaunchKernelEx(&cfg, gemm_int4_kernel, ta, tb, tz, tl2, ty, tsa, tsb, p);
+  cfg.numAttrs = split ? 2 : 1;
+  e = split ? cudaLaunchKernelEx(&cfg, gemm_int4_kernel<true>, ta, tb, tz, tl2, ty, tsa, tsb, q)
+            : cudaLaunchKernelEx(&cfg, gemm_int4_kernel<false>, ta, tb, tz, tl2, ty, tsa, tsb, q);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

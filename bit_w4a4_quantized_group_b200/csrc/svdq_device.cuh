@@ -142,6 +142,7 @@ struct GemmParams {
   int num_tiles, tiles_m, tiles_n;
   int op_pair;               // FP4: A and B tensor maps are 3-D and load two K steps at once
   int y_align32;             // Y is 32-byte aligned (256-bit stores)
+  int ksplit;                // INT4: CTAs of a cluster that split one tile's K steps (1: none)
 };
 
 cudaError_t launch_prologue(int fmt, const CUtensorMap& tx, const CUtensorMap& tl1, const ProParams& p,
