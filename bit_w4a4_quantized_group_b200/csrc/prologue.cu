@@ -26,7 +26,10 @@
 // the first forms X_hat, the Z products and the row maxima; the compute warps then
 // combine their maxima and write the fp32 row scales; the second pass re-reads X (the
 // CTAs' rows were just read, so the L2 serves most of it), re-forms X_hat and writes
-// one-byte codes with an IEEE-exact divide by the row scale.
+// one-byte codes with an IEEE-exact divide by the row scale.  Under the K split each CTA
+// publishes its rows' maxima after the first pass and signals every peer of the cluster
+// (a remote mbarrier arrive with release at cluster scope); once all peers have signalled,
+// it takes the maximum over the cluster (exact, order-independent) before the second pass.
 //
 // Divisions are IEEE-exact without the divide instruction sequence:
 //  * X / lambda uses Markstein's correction (P. Markstein, "Computation of
@@ -142,7 +145,9 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   constexpr int NPASS = passes(FMT);
   uint8_t* cstage = reinterpret_cast<uint8_t*>(empty + S);          // NW warps x CSTB code staging
   float* rmax_s = reinterpret_cast<float*>(cstage + NW * CSTB);     // W8A8: [BOXES][2 strips][16 rows]
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(rmax_s + BOXES * 32);
+  float* rmax_cta = rmax_s + BOXES * 32;                              // W8A8 K split: this CTA's 32 row maxima
+  uint64_t* rm_bar = reinterpret_cast<uint64_t*>(rmax_cta + 32);      // ... published by every peer
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(rm_bar + 1);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -162,10 +167,13 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       ptx::mbar_init(&full[s], 32);     // every producer lane arrives (its lambda stores) + TMA bytes
       ptx::mbar_init(&empty[s], NW);
     }
+    if (SPLIT && FMT == kFmtW8a8) ptx::mbar_init(rm_bar, static_cast<uint32_t>(p.ksplit - 1));
     *abort_flag = 0;
     ptx::fence_mbar_init();
   }
   __syncthreads();
+  // W8A8 K split: every CTA's barriers are initialised before any peer can arrive on them
+  if (SPLIT && FMT == kFmtW8a8) ptx::cluster_sync();
   // the GEMM launched after this kernel may start its own set-up now (on SMs this grid leaves
   // free); it reads this kernel's outputs only after the whole grid has completed
   ptx::griddep_launch_dependents();
@@ -530,9 +538,34 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
       }
       // s = RN_f32(a / 127): the fp64 quotient rounded to fp32 is the correctly rounded fp32
       // quotient (53 >= 2 * 24 + 2 bits, so the double rounding is innocuous)
+      if (SPLIT) {
+        // K split: the scale needs the row maximum over all of K, i.e. over the cluster.  Every
+        // CTA publishes its 32 rows' maxima and signals every peer (release at cluster scope);
+        // after all peers have signalled, it takes the maximum of all CTAs' values (exact and
+        // order-independent: every CTA derives the same scales)
+        if (phase == 0 && tig == 0) {
+          rmax_cta[strip * 16 + g] = amax_a;
+          rmax_cta[strip * 16 + g + 8] = amax_b;
+        }
+        named_barrier_sync(2, 32 * NW);
+        if (warp == 0 && lane == 0) {
+          for (int q = 0; q < p.ksplit; ++q)
+            if (q != split) ptx::mbar_arrive_cluster(ptx::mapa_shared(ptx::smem_u32(rm_bar), static_cast<uint32_t>(q)));
+        }
+        if (!wait_bounded(rm_bar, 0u, abort_flag, p.err, kErrSiteProFull)) ok = false;
+        ptx::fence_acq_rel_cluster();
+        if (ok) {
+          const uint32_t ra = ptx::smem_u32(rmax_cta + strip * 16 + g), rb2 = ptx::smem_u32(rmax_cta + strip * 16 + g + 8);
+          for (int q = 0; q < p.ksplit; ++q) {
+            if (q == split) continue;
+            amax_a = fmaxf(amax_a, ptx::ld_shared_cluster_f32(ptx::mapa_shared(ra, static_cast<uint32_t>(q))));
+            amax_b = fmaxf(amax_b, ptx::ld_shared_cluster_f32(ptx::mapa_shared(rb2, static_cast<uint32_t>(q))));
+          }
+        }
+      }
       const float sa = __double2float_rn(__ddiv_rn(static_cast<double>(amax_a), 127.0));
       const float sb = __double2float_rn(__ddiv_rn(static_cast<double>(amax_b), 127.0));
-      if (phase == 0 && tig == 0) {
+      if (phase == 0 && tig == 0 && split == 0) {
         float* sc = reinterpret_cast<float*>(p.scales);
         if (SVDQ_IN_GLOBAL(row_b < p.Mpad, p.err)) {
           sc[row_a] = sa;             // rows up to Mpad; rows past M read zeros and get 0
@@ -594,10 +627,10 @@ __global__ void __launch_bounds__(32 * (compute_warps(RANK) + 1), 1)
   // K split over a cluster: CTA 0 adds the other CTAs' Z partials (read through distributed
   // shared memory, in CTA order) and writes Z.  Every thread of every CTA reaches both
   // cluster barriers; a wait that ran out above only ends its loop early.
-  if (RANK > 0 && SPLIT) {
+  if (SPLIT && (RANK > 0 || FMT == kFmtW8a8)) {
     constexpr int R1 = RANK > 0 ? RANK : 1;
     ptx::cluster_sync();                                      // every partial is in shared memory
-    if (split == 0) {
+    if (RANK > 0 && split == 0) {
       // every thread of CTA 0 takes two columns of the 32 x RANK block: the peers' partials
       // are all requested before any is added (remote reads overlap), then added in CTA order
       constexpr int kMaxSplit = 8;
@@ -641,14 +674,14 @@ size_t smem_bytes_for(int stages) {
   constexpr int NW = compute_warps(RANK);
   const ProSmemLayout L = pro_layout(RANK, NW / 2);
   return 1024 + static_cast<size_t>(stages) * L.stage_bytes + 2 * stages * 8 + NW * code_stage_bytes(FMT) +
-         (NW / 2) * 32 * 4 + 16;
+         (NW / 2) * 32 * 4 + 32 * 4 + 8 + 16;
 }
 
 template <int FMT, int RANK>
 int stages_for() {
   constexpr int NW = compute_warps(RANK);
   const ProSmemLayout L = pro_layout(RANK, NW / 2);
-  const size_t budget = 220 * 1024 - 1024 - NW * code_stage_bytes(FMT) - (NW / 2) * 32 * 4 - 64;
+  const size_t budget = 220 * 1024 - 1024 - NW * code_stage_bytes(FMT) - (NW / 2) * 32 * 4 - 32 * 4 - 8 - 64;
   int s = static_cast<int>(budget / L.stage_bytes);
   if (s > 4) s = 4;
   return s;
@@ -706,7 +739,7 @@ static cudaError_t launch_pro(const CUtensorMap& tx, const CUtensorMap& tl1, Pro
   if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
     return cudaErrorInvalidDevice;
   p.ksplit = 1;
-  if (FMT != kFmtW8a8) {
+  {
     for (int ks = 8; ks >= 2; --ks) {
       const int nks = (nkt_all + ks - 1) / ks;
       if (ks <= nkt_all && nks * (ks - 1) < nkt_all && blocks * ks <= sms &&

@@ -446,13 +446,13 @@ def test_layer_random_shapes(case):
                                                              packed["L2_bf16"] if rank else None, layer.bias))
 
 
-@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4"])
+@pytest.mark.parametrize("fmt", ["nvfp4", "int4", "mxfp4", "w8a8"])
 @pytest.mark.parametrize("M,K,N,rank", [(256, 3072, 3072, 32), (1024, 3072, 1024, 64), (40, 2048, 512, 16),
                                         (256, 12288, 512, 32)])
 def test_layer_small_batch_k_split(fmt, M, K, N, rank):
     """Small batches, where the prologue splits each row block's K stages over a cluster of
-    CTAs and adds their Z partials through distributed shared memory; the whole layer
-    against the reference."""
+    CTAs and adds their Z partials through distributed shared memory (W8A8: after taking each
+    row's maximum over the cluster); the whole layer against the reference."""
     layer, prep = _layer(M, K, N, rank, seed=77 + M + rank, fmt=fmt)
     gx = prep["act_gscale"]
     pk = B.pack_weight_np(fmt, prep["R_nk"].astype(np.float32), prep["L1_rk"].astype(np.float32),
